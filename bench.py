@@ -1,0 +1,368 @@
+"""Benchmark of the fused chunked KL loss (forward + backward) on B200.
+
+    python bench.py [--gpus N --steps K --warmup W] [--config 8b|small|tiny|large_vocab|sweep] [--N n]
+    python bench.py --impl reference ...      # the CPU oracle on a bounded sample (baseline arm)
+
+One step = kdkl_forward + kdkl_backward over one batch of seeded synthetic
+inputs already resident in HBM.  Rank 0 prints one JSON line.  With N > 1
+(torchrun) every rank runs an independent replica on its own seeded batch
+(replicas only: the library is single-GPU; no collective on the data path)
+and `value` is the tokens of all ranks divided by the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "fused KL fwd+bwd tokens/sec and % of B200 bf16 tensor peak; peak GB vs N"
+UNIT = "tokens/s"
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"bf16_tflops": float(d["bf16_tflops"]), "bf16_tflops_sustained": float(d["bf16_tflops_sustained"]),
+                "hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- clocks
+_REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+                0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+                0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms while the timed region runs."""
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        cmd = ["nvidia-smi", "-i", self.gpu_id,
+               "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
+               "--format=csv,noheader,nounits", "-lms", "200"]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.t:
+            self.t.join(timeout=5)
+        sm, smax, reasons = [], [], set()
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 4:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+                mask = int(parts[3], 16)
+            except ValueError:
+                continue
+            for bit, name in _REASON_BITS.items():
+                if mask & bit and name != "gpu_idle":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        busy = [s for s in sm if s > 0.3 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def gpu_id_for(dev_index: int) -> str:
+    import torch
+    props = torch.cuda.get_device_properties(dev_index)
+    uuid = getattr(props, "uuid", None)
+    if uuid is not None:
+        s = str(uuid)
+        return s if s.startswith("GPU-") else "GPU-" + s
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        return vis.split(",")[dev_index]
+    return str(dev_index)
+
+
+# ----------------------------------------------------------------------------- oracle arm
+def oracle_sample(x: synth.Inputs, rows: int, seed: int):
+    """Times the CPU oracle (as it stands) on a bounded sample of the workload's rows."""
+    from oracle import kl as O
+    sel = synth.sample_rows(x.hidden_bits.shape[0], rows, seed)
+    sub = (x.hidden_bits[sel], x.W_bits, x.topk_idx[sel], x.topk_logit[sel], x.mask[sel], x.tau)
+    t0 = time.perf_counter()
+    O.kl_loss(*sub)
+    dt = time.perf_counter() - t0
+    return sel.size, dt
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = [i.get("num_threads", 0) for i in info if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def sample_rows_for(w: synth.Workload, target_s: float = 15.0) -> int:
+    # oracle cost per row ~ 3 * 2 d V fp64 flops (logits, dHidden, dW) plus O(V) elementwise work
+    per_row = 6.0 * w.d * w.V / 2.0e11 + w.V * 2.0e-7
+    return int(max(16, min(4096, target_s / per_row)))
+
+
+def run_reference(args, w: synth.Workload, N: int):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    x = synth.make_inputs(w, N=N)
+    rows = sample_rows_for(w, target_s=max(2.0, 60.0 / max(1, args.steps + args.warmup)))
+    for i in range(args.warmup):
+        oracle_sample(x, rows, seed=1000 + i)
+    times = []
+    for i in range(args.steps):
+        n, dt = oracle_sample(x, rows, seed=2000 + i)
+        times.append(dt)
+    total = sum(times)
+    value = rows * args.steps / total
+    cores = blas_threads()
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1000.0 * total / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": w.name, "N": N, "d": w.d, "V": w.V, "K": w.K, "tau": w.tau,
+                       "sample_rows_per_step": rows},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"{rows} seeded rows of the {w.name} workload per step, full fwd+bwd "
+                                       f"(loss, lse, dHidden, dW contribution) in numpy float64"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def main_gpu(args, w: synth.Workload, N: int):
+    import torch
+    import torch.distributed as dist
+
+    import output_head_kl_b200 as K
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=dev)
+
+    K.lib()
+    t_gen = time.perf_counter()
+    x = synth.make_inputs(w, N=N, seed=synth.seed_for(w, N) + 7919 * rank)
+    t_gen = time.perf_counter() - t_gen
+    Nn, d, V, Kc = x.shape
+
+    def bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+
+    h_hidden = bf16(x.hidden_bits).pin_memory()
+    h_idx = torch.from_numpy(x.topk_idx).pin_memory()
+    h_logit = torch.from_numpy(x.topk_logit).pin_memory()
+    h_mask = torch.from_numpy(x.mask).pin_memory()
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats(dev)
+    base_alloc = torch.cuda.memory_allocated(dev)
+    W = bf16(x.W_bits).to(dev)
+
+    hidden = h_hidden.to(dev)
+    idx = h_idx.to(dev)
+    logit = h_logit.to(dev)
+    mask = h_mask.to(dev)
+    ws_bytes = K.kdkl_workspace_bytes(Nn, d, V, Kc, args.chunk_tokens)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    lse = torch.empty(Nn, dtype=torch.float32, device=dev)
+    dH = torch.empty(Nn, d, dtype=torch.bfloat16, device=dev)
+    dW = torch.empty(V, d, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        K.kdkl_forward(hidden, W, idx, logit, mask, x.tau, loss, lse, ws, stream=stream)
+        K.kdkl_backward(hidden, W, idx, logit, mask, x.tau, lse, None, dH, dW, ws,
+                        chunk_tokens=args.chunk_tokens, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    flags = K.kdkl_read_device_flags(ws)
+    peak_bytes = torch.cuda.max_memory_allocated(dev) - base_alloc
+    K.kdkl_timing_read(reset=True)
+
+    sampler = ClockSampler(gpu_id_for(local)) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    K.kdkl_timing_enable(True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    K.kdkl_timing_enable(False)
+    kt = K.kdkl_timing_read(reset=True)
+    clocks = sampler.stop() if sampler else None
+    ms = e0.elapsed_time(e1) / args.steps
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+
+    # end-to-end through the public API with host buffers: per step the batch
+    # (hidden, cache, mask) goes host -> device from pinned memory and the
+    # loss comes back device -> host
+    h_loss = torch.empty(1, dtype=torch.float32).pin_memory()
+    e2e_steps = max(1, min(args.steps, 5))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(e2e_steps):
+        hidden.copy_(h_hidden, non_blocking=True)
+        idx.copy_(h_idx, non_blocking=True)
+        logit.copy_(h_logit, non_blocking=True)
+        mask.copy_(h_mask, non_blocking=True)
+        step()
+        h_loss.copy_(loss, non_blocking=True)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([t0.elapsed_time(t1) / e2e_steps], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_ms = float(e2e_ms.item())
+    h2d = Nn * d * 2 + Nn * Kc * 4 * 2 + Nn
+    d2h = 4
+
+    out = None
+    if rank == 0:
+        peaks = measured_peaks()
+        flops = synth.flops_fwd_bwd(Nn, d, V)
+        tflops = flops / (ms_max * 1e-3) / 1e12
+        # dominant kernel by total time; its algorithmic flops are 2 N d V per step
+        gemm_kinds = ("fwd_lse_gemm", "bwd_grad_gemm", "bwd_dhidden_gemm", "bwd_dw_gemm")
+        dom = max(kt, key=lambda k: kt[k][1])
+        launches, total_ms = kt[dom]
+        if dom in gemm_kinds and launches:
+            alg = 2.0 * Nn * d * V * args.steps / launches
+            achieved = alg / (total_ms / launches * 1e-3) / 1e12
+            roof = {"kernel": dom, "bound": "tensor", "achieved": achieved,
+                    "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                    "frac": achieved / peaks["bf16_tflops_sustained"],
+                    "peak_kind": f"bf16 dense, sustained ({peaks['source']})",
+                    "frac_of_burst_peak": achieved / peaks["bf16_tflops"],
+                    "flops_per_launch": alg, "avg_launch_ms": total_ms / launches,
+                    "traffic": None}
+        else:
+            roof = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": None, "traffic": None}
+        kernels = {k: {"launches": v[0], "ms_per_step": v[1] / args.steps} for k, v in kt.items() if v[0]}
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            rows = sample_rows_for(w)
+            n_rows, dt = oracle_sample(x, rows, seed=4242)
+            cpu = {"value": n_rows / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                   "sample": f"{n_rows} seeded rows of the {w.name} workload, one full fwd+bwd "
+                             f"(loss, lse, dHidden, dW contribution) in numpy float64, {dt:.1f} s"}
+        out = {
+            "metric": METRIC, "value": Nn * world / (ms_max * 1e-3), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "N": Nn, "d": d, "V": V, "K": Kc, "tau": x.tau,
+                       "chunk_tokens": args.chunk_tokens or min(8192, (Nn + 127) // 128 * 128),
+                       "l2": "inputs larger than L2 (W alone is %.2f GB); no flush" % (V * d * 2 / 1e9),
+                       "parallelism": f"replicas x{world}"},
+            "tflops": tflops,
+            "frac_of_bf16_peak": tflops / peaks["bf16_tflops"],
+            "frac_of_bf16_peak_sustained": tflops / peaks["bf16_tflops_sustained"],
+            "peak_gb": peak_bytes / 1e9,
+            "workspace_gb": ws_bytes / 1e9,
+            "roofline": roof,
+            "kernels": kernels,
+            "cpu_baseline": cpu,
+            "e2e": {"value": Nn * world / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": int(sum(v[0] for v in kt.values())),
+            "clocks": clocks,
+            "device_flags": flags,
+            "input_gen_s": t_gen,
+        }
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="kdkl", choices=["kdkl", "reference"])
+    ap.add_argument("--config", default="8b", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--N", type=int, default=None, help="token count override (sweep points)")
+    ap.add_argument("--chunk-tokens", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = synth.CONFIGS[args.config]
+    N = args.N if args.N is not None else w.N
+    if args.impl == "reference":
+        return run_reference(args, w, N)
+    return main_gpu(args, w, N)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,153 @@
+/*
+ * kdkl — fused, chunked KL distillation loss of a student output head against
+ * an offline teacher top-K cache, for one NVIDIA B200 (sm_100a).
+ *
+ * Method: "Efficient Knowledge Distillation for LLMs: Offline Top-K Logits and
+ * a Fused Chunked KL Loss".  The teacher is run once and only its top-K
+ * (vocabulary index, logit) pairs per token are kept (mind-verse.de article,
+ * section "Zwei systemische Optimierungen", item 1; llm-wiki note, section
+ * "사전 계산 파이프라인", step 3).  The loss folds the student's output
+ * projection into the KL computation and never holds the full
+ * [tokens x vocabulary] logit matrix; the backward recomputes each chunk's
+ * projection (mind-verse.de article, three-variant list, "Fused chunked KL").
+ *
+ * Definitions (N tokens, hidden size d, vocabulary V, K cached entries, tau):
+ *   z[n, v]   = sum_j hidden[n, j] * W[v, j]              (student logits)
+ *   lse[n]    = log sum_v exp(z[n, v])
+ *   P_T[n, .] = softmax(topk_logit[n, .] / tau) over the row's in-range entries,
+ *               zero on every other vocabulary entry
+ *   KL_n      = sum_v P_T(v) (log P_T(v) - (z[n, v] - lse[n]))
+ *               (llm-wiki note, section "표준 KD의 손실 함수")
+ *   loss      = sum_n m_n KL_n / N_valid,  m_n = mask[n] and the row is usable,
+ *               N_valid = sum_n m_n  (loss = 0 when N_valid = 0)
+ *   G[n, v]   = m_n (g / N_valid) (exp(z[n, v] - lse[n]) - P_T[n](v))
+ *   dHidden   = G W   [N, d],   dW = G^T hidden   [V, d]
+ * tau divides the teacher logits only (there is no tau^2 factor).
+ *
+ * Conventions for every entry point below:
+ *   - All tensors are dense, row-major, on the current CUDA device, and owned
+ *     by the caller.  The library never allocates device memory: scratch comes
+ *     from the caller's `workspace`.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL
+ *     is the legacy default stream).  Nothing synchronises except
+ *     kdkl_read_device_flags.  No state is kept between calls.
+ *   - Argument checks run on the host before any launch; a failed check
+ *     returns its status and launches nothing.  kdkl_last_error() then holds a
+ *     one-line reason.
+ *   - Data errors found on the device (cache index outside [0, V), repeated
+ *     index, non-finite teacher logit, an internal wait that timed out) never
+ *     trap: they set bits of a device flag word kept in the workspace, which
+ *     the caller reads with kdkl_read_device_flags.  Entries with an index
+ *     outside [0, V) are dropped; repeated indices add up; a row with a NaN or
+ *     +inf logit, or with no usable entry, is treated as masked.
+ */
+#ifndef KDKL_H
+#define KDKL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KDKL_OK = 0,
+  KDKL_ERR_NULL = 1,        /* a required pointer is NULL */
+  KDKL_ERR_SHAPE = 2,       /* N < 0, d % 8 != 0, K outside [1, 256], K > V, tau not finite > 0, ... */
+  KDKL_ERR_ALIGN = 3,       /* a pointer breaks its alignment rule (listed per argument) */
+  KDKL_ERR_UNSUPPORTED = 4, /* no sm_100 device current, or a size beyond the library's limits */
+  KDKL_ERR_WORKSPACE = 5,   /* workspace smaller than kdkl_workspace_bytes() */
+  KDKL_ERR_CUDA = 6         /* a CUDA runtime call or launch failed */
+} kdkl_status;
+
+/* Bits of the device flag word (kdkl_read_device_flags). */
+enum {
+  KDKL_DEV_IDX_RANGE = 1u, /* some cached index was outside [0, V); the entry was dropped */
+  KDKL_DEV_IDX_DUP = 2u,   /* some row repeated a cached index; the probabilities were added */
+  KDKL_DEV_NONFINITE = 4u, /* some row had a NaN/+inf (or only -inf) logit; the row was masked */
+  KDKL_DEV_TIMEOUT = 8u    /* an internal pipeline wait gave up; this call's outputs are invalid */
+};
+
+/*
+ * Bytes of scratch that kdkl_forward / kdkl_backward need for these sizes.
+ * The amount is linear in N plus one N-independent chunk buffer of
+ * chunk_tokens x V bf16 values (the backward's per-chunk logit gradient); it
+ * never holds an N x V buffer.  chunk_tokens = 0 picks the library default
+ * (min(N rounded up to 128, 8192)); other values are rounded up to a multiple
+ * of 128.  Returns 0 for sizes that the entry points would reject.
+ */
+size_t kdkl_workspace_bytes(int64_t N, int32_t d, int32_t V, int32_t K, int64_t chunk_tokens);
+
+/*
+ * Forward: loss and per-token log-sum-exp.
+ *   hidden      [N, d] bf16, 16-byte aligned (student last hidden states)
+ *   W           [V, d] bf16, 16-byte aligned (output-head weight, nn.Linear layout, no bias)
+ *   topk_idx    [N, K] int32, 4-byte aligned (teacher cache: vocabulary indices)
+ *   topk_logit  [N, K] fp32, 4-byte aligned (teacher cache: logits)
+ *   mask        [N] uint8 (0 = token excluded, e.g. a packed-sequence boundary)
+ *   N >= 0, d % 8 == 0 (d >= 8), 1 <= K <= 256, K <= V, tau finite and > 0
+ *   loss        [1] fp32 out (device), 4-byte aligned
+ *   lse         [N] fp32 out (device), 4-byte aligned; written for every row, masked ones too
+ *   workspace   >= kdkl_workspace_bytes(N, d, V, K, 0) bytes, 256-byte aligned
+ * N = 0 writes loss = 0 and nothing else.
+ */
+kdkl_status kdkl_forward(const void* hidden, const void* W, const int32_t* topk_idx,
+                         const float* topk_logit, const uint8_t* mask, int64_t N, int32_t d,
+                         int32_t V, int32_t K, float tau, float* loss, float* lse,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Backward: dHidden and dW of g * loss, recomputing each chunk's projection.
+ *   inputs as kdkl_forward, plus
+ *   lse          [N] fp32 in: the lse written by kdkl_forward on the same inputs
+ *   grad_loss    [1] fp32 in (device) = g, or NULL for g = 1
+ *   dHidden      [N, d] bf16 out, 16-byte aligned (fp32 accumulation, rounded once);
+ *                rows that do not count (masked or unusable) are written as 0
+ *   dW           [V, d] fp32 out, 16-byte aligned, overwritten (not accumulated into)
+ *   chunk_tokens tokens per backward chunk (0 = default); bounds the chunk buffer
+ *   workspace    >= kdkl_workspace_bytes(N, d, V, K, chunk_tokens) bytes, 256-byte aligned
+ * N = 0 writes dW = 0 and nothing else.
+ */
+kdkl_status kdkl_backward(const void* hidden, const void* W, const int32_t* topk_idx,
+                          const float* topk_logit, const uint8_t* mask, int64_t N, int32_t d,
+                          int32_t V, int32_t K, float tau, const float* lse,
+                          const float* grad_loss, void* dHidden, float* dW,
+                          int64_t chunk_tokens, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/*
+ * Reads the device flag word of the most recent forward/backward call that
+ * used `workspace` (each call clears it first).  Synchronises `stream`.
+ */
+kdkl_status kdkl_read_device_flags(const void* workspace, void* stream, uint32_t* flags_out);
+
+/*
+ * Optional per-kernel timing (tracing aid; off by default).  While enabled,
+ * every kernel the library launches is bracketed by a pair of CUDA events
+ * recorded on the caller's stream, tagged with the kernel's name.
+ * kdkl_timing_read waits for the pending events, adds their durations into
+ * per-kernel totals, copies up to max_entries totals into `out` (names are
+ * static strings) and returns how many kernel kinds exist; reset != 0 clears
+ * the totals afterwards.  Enabling costs two event records per launch.
+ */
+typedef struct {
+  const char* name;   /* "prepass", "fwd_lse_gemm", "merge", "bwd_grad_gemm", "bwd_dhidden_gemm", "bwd_dw_gemm" */
+  uint64_t launches;  /* launches timed since the last reset */
+  double total_ms;    /* summed device time of those launches */
+} kdkl_kernel_time;
+
+kdkl_status kdkl_timing_enable(int enable);
+int kdkl_timing_read(kdkl_kernel_time* out, int max_entries, int reset);
+
+/* Static name of a status code. */
+const char* kdkl_status_string(kdkl_status status);
+
+/* One-line reason for the last non-OK status returned on this host thread ("" if none). */
+const char* kdkl_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDKL_H */

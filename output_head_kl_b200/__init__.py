@@ -1,0 +1,175 @@
+"""Python binding of the kdkl C ABI (``include/kdkl.h``): argument marshalling only.
+
+Every step of the loss runs in the CUDA library ``_lib/libkdkl.so``; this module
+turns torch tensors into pointers and status codes into exceptions.  There is
+no fallback: if the library is missing, importing a function that needs it
+raises.
+
+Names mirror the C entry points: ``kdkl_workspace_bytes``, ``kdkl_forward``,
+``kdkl_backward``, ``kdkl_read_device_flags``, ``kdkl_timing_enable``,
+``kdkl_timing_read``, ``kdkl_status_string``, ``kdkl_last_error``.  ``fused_kl_forward_backward`` is a convenience wrapper
+that allocates the outputs and the workspace with torch (the library itself
+never allocates).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_lib", "libkdkl.so")
+
+KDKL_OK = 0
+STATUS_NAMES = {0: "KDKL_OK", 1: "KDKL_ERR_NULL", 2: "KDKL_ERR_SHAPE", 3: "KDKL_ERR_ALIGN",
+                4: "KDKL_ERR_UNSUPPORTED", 5: "KDKL_ERR_WORKSPACE", 6: "KDKL_ERR_CUDA"}
+DEV_IDX_RANGE, DEV_IDX_DUP, DEV_NONFINITE, DEV_TIMEOUT = 1, 2, 4, 8
+
+_lib = None
+
+
+class KernelTime(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char_p), ("launches", ctypes.c_uint64), ("total_ms", ctypes.c_double)]
+
+
+class KDKLError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}: {detail}")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """Loads the in-tree CUDA library (raises if it was not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"kdkl CUDA library not built: {LIB_PATH} is missing "
+                           "(run `python -m output_head_kl_b200.build`)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32, f32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    L.kdkl_workspace_bytes.argtypes = [i64, i32, i32, i32, i64]
+    L.kdkl_workspace_bytes.restype = sz
+    L.kdkl_forward.argtypes = [vp, vp, vp, vp, vp, i64, i32, i32, i32, f32, vp, vp, vp, sz, vp]
+    L.kdkl_forward.restype = ctypes.c_int
+    L.kdkl_backward.argtypes = [vp, vp, vp, vp, vp, i64, i32, i32, i32, f32, vp, vp, vp, vp, i64, vp, sz, vp]
+    L.kdkl_backward.restype = ctypes.c_int
+    L.kdkl_read_device_flags.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
+    L.kdkl_read_device_flags.restype = ctypes.c_int
+    L.kdkl_status_string.argtypes = [ctypes.c_int]
+    L.kdkl_status_string.restype = ctypes.c_char_p
+    L.kdkl_last_error.argtypes = []
+    L.kdkl_last_error.restype = ctypes.c_char_p
+    L.kdkl_timing_enable.argtypes = [ctypes.c_int]
+    L.kdkl_timing_enable.restype = ctypes.c_int
+    L.kdkl_timing_read.argtypes = [ctypes.POINTER(KernelTime), ctypes.c_int, ctypes.c_int]
+    L.kdkl_timing_read.restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int, where: str):
+    if status != KDKL_OK:
+        raise KDKLError(status, where, kdkl_last_error())
+
+
+def kdkl_status_string(status: int) -> str:
+    return lib().kdkl_status_string(status).decode()
+
+
+def kdkl_last_error() -> str:
+    return lib().kdkl_last_error().decode()
+
+
+def kdkl_workspace_bytes(N: int, d: int, V: int, K: int, chunk_tokens: int = 0) -> int:
+    return int(lib().kdkl_workspace_bytes(N, d, V, K, chunk_tokens))
+
+
+def kdkl_forward(hidden, W, topk_idx, topk_logit, mask, tau, loss, lse, workspace, *, N=None, d=None, V=None,
+                 K=None, workspace_bytes=None, stream=None, check=True) -> int:
+    """Calls kdkl_forward.  Tensors (or raw device pointers with explicit sizes)."""
+    N = hidden.shape[0] if N is None else N
+    d = hidden.shape[1] if d is None else d
+    V = W.shape[0] if V is None else V
+    K = topk_idx.shape[1] if K is None else K
+    wsb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    st = lib().kdkl_forward(_ptr(hidden), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask), int(N), int(d),
+                            int(V), int(K), float(tau), _ptr(loss), _ptr(lse), _ptr(workspace), int(wsb),
+                            _stream(stream))
+    if check:
+        _check(st, "kdkl_forward")
+    return st
+
+
+def kdkl_backward(hidden, W, topk_idx, topk_logit, mask, tau, lse, grad_loss, dHidden, dW, workspace, *,
+                  chunk_tokens=0, N=None, d=None, V=None, K=None, workspace_bytes=None, stream=None,
+                  check=True) -> int:
+    """Calls kdkl_backward (grad_loss may be None for g = 1)."""
+    N = hidden.shape[0] if N is None else N
+    d = hidden.shape[1] if d is None else d
+    V = W.shape[0] if V is None else V
+    K = topk_idx.shape[1] if K is None else K
+    wsb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    st = lib().kdkl_backward(_ptr(hidden), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask), int(N), int(d),
+                             int(V), int(K), float(tau), _ptr(lse), _ptr(grad_loss), _ptr(dHidden), _ptr(dW),
+                             int(chunk_tokens), _ptr(workspace), int(wsb), _stream(stream))
+    if check:
+        _check(st, "kdkl_backward")
+    return st
+
+
+def kdkl_read_device_flags(workspace, stream=None) -> int:
+    out = ctypes.c_uint32(0)
+    _check(lib().kdkl_read_device_flags(_ptr(workspace), _stream(stream), ctypes.byref(out)),
+           "kdkl_read_device_flags")
+    return int(out.value)
+
+
+def kdkl_timing_enable(enable: bool = True) -> None:
+    _check(lib().kdkl_timing_enable(1 if enable else 0), "kdkl_timing_enable")
+
+
+def kdkl_timing_read(reset: bool = False) -> dict:
+    """{kernel name: (launches, total ms)} accumulated since the last reset."""
+    arr = (KernelTime * 16)()
+    n = lib().kdkl_timing_read(arr, 16, 1 if reset else 0)
+    return {arr[i].name.decode(): (int(arr[i].launches), float(arr[i].total_ms)) for i in range(n)}
+
+
+def fused_kl_forward_backward(hidden, W, topk_idx, topk_logit, mask, tau, *, grad_loss=None, chunk_tokens=0,
+                              workspace=None, stream=None):
+    """Forward + backward with torch-allocated outputs.
+
+    Returns (loss[1] f32, lse[N] f32, dHidden[N, d] bf16, dW[V, d] f32, workspace).
+    """
+    import torch
+    N, d = hidden.shape
+    V = W.shape[0]
+    K = topk_idx.shape[1]
+    dev = hidden.device
+    if workspace is None:
+        workspace = torch.empty(kdkl_workspace_bytes(N, d, V, K, chunk_tokens), dtype=torch.uint8, device=dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    lse = torch.empty(N, dtype=torch.float32, device=dev)
+    dH = torch.empty(N, d, dtype=torch.bfloat16, device=dev)
+    dW = torch.empty(V, d, dtype=torch.float32, device=dev)
+    kdkl_forward(hidden, W, topk_idx, topk_logit, mask, tau, loss, lse, workspace, stream=stream)
+    kdkl_backward(hidden, W, topk_idx, topk_logit, mask, tau, lse, grad_loss, dH, dW, workspace,
+                  chunk_tokens=chunk_tokens, stream=stream)
+    return loss, lse, dH, dW, workspace

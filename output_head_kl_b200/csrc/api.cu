@@ -1,0 +1,505 @@
+// C ABI of the fused chunked KL loss: argument checks, workspace layout,
+// work planner, TMA descriptors and the token-chunk scheduler of the backward.
+//
+// The forward needs no token chunking: its per-row state (running max,
+// sum-exp, gathered logit) is O(N), and the vocabulary is swept tile by tile
+// with an online log-sum-exp (the vocabulary-axis chunking of the llm-wiki
+// note, section "Fused Chunked KL").  The backward loops over token chunks
+// (the sequence-axis chunking of the mind-verse.de article, three-variant list,
+// "Fused chunked KL"): each chunk's logits are recomputed, turned into the
+// gradient G on chip, written once as bf16 into an N-independent chunk buffer,
+// and consumed by the dHidden and dW GEMMs before the next chunk overwrites it.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/kdkl.h"
+#include "kdkl_internal.h"
+
+namespace kdkl {
+namespace {
+
+thread_local char g_last_error[256] = {0};
+
+kdkl_status fail(kdkl_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+kdkl_status ok() {
+  g_last_error[0] = 0;
+  return KDKL_OK;
+}
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+constexpr int64_t kDefaultChunk = 8192;
+constexpr int64_t kMaxRows = (int64_t(1) << 31) - 256;
+constexpr int32_t kMaxV = (int32_t(1) << 30);
+
+// --------------------------------------------------------------- tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 map: `inner` contiguous elements per row, `outer` rows, row pitch in elements.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t pitch_elems,
+              uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {pitch_elems * 2};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// --------------------------------------------------------------- planner
+struct Device {
+  int id = 0;
+  int sms = 0;
+  int cc_major = 0;
+};
+
+kdkl_status current_device(Device& dv) {
+  if (cudaGetDevice(&dv.id) != cudaSuccess) return fail(KDKL_ERR_UNSUPPORTED, "no CUDA device is current");
+  if (cudaDeviceGetAttribute(&dv.sms, cudaDevAttrMultiProcessorCount, dv.id) != cudaSuccess ||
+      cudaDeviceGetAttribute(&dv.cc_major, cudaDevAttrComputeCapabilityMajor, dv.id) != cudaSuccess)
+    return fail(KDKL_ERR_CUDA, "cudaDeviceGetAttribute failed");
+  if (dv.cc_major != 10) return fail(KDKL_ERR_UNSUPPORTED, "kdkl needs an sm_100 device (found cc %d.x)", dv.cc_major);
+  return KDKL_OK;
+}
+
+// Vocabulary splits for a row-stream kernel over `rb` row blocks and `vt`
+// vocabulary tiles: balance the per-CTA tile count over `ctas`, and keep at
+// least enough splits that the hidden rows in flight stay small next to L2.
+int pick_splits(int64_t rb, int vt, int ctas, int d, int64_t units_cap) {
+  const double rows_bytes = 128.0 * d * 2.0;
+  const double budget = 48.0 * 1024 * 1024;
+  int s_min = static_cast<int>(std::ceil(ctas * rows_bytes / budget));
+  if (s_min < 1) s_min = 1;
+  int s_max = static_cast<int>(units_cap / rb);
+  if (s_max > vt) s_max = vt;
+  if (s_max < 1) s_max = 1;
+  if (s_min > s_max) s_min = s_max;
+  int best = s_min;
+  double best_cost = 1e300;
+  for (int s = s_min; s <= s_max; ++s) {
+    const int64_t units = rb * s;
+    const int64_t waves = (units + ctas - 1) / ctas;
+    const int64_t per_unit = (vt + s - 1) / s;
+    // small per-unit overhead term favours fewer, longer units on ties
+    const double cost = static_cast<double>(waves * per_unit) + 0.01 * waves;
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
+}
+
+int pick_bn(int d) {
+  // smallest padded width; ties go to the wider tile
+  const int cands[3] = {256, 192, 128};
+  int best = 256;
+  int64_t best_pad = INT64_MAX;
+  for (int c : cands) {
+    const int64_t pad = static_cast<int64_t>((d + c - 1) / c) * c;
+    if (pad < best_pad) {
+      best_pad = pad;
+      best = c;
+    }
+  }
+  return best;
+}
+
+kdkl_status check_shapes(int64_t N, int32_t d, int32_t V, int32_t K, float tau) {
+  if (N < 0 || N > kMaxRows) return fail(KDKL_ERR_SHAPE, "N=%lld outside [0, %lld]", (long long)N, (long long)kMaxRows);
+  if (d < 8 || d % 8 != 0) return fail(KDKL_ERR_SHAPE, "d=%d must be a positive multiple of 8", d);
+  if (V < 1 || V > kMaxV) return fail(KDKL_ERR_SHAPE, "V=%d outside [1, 2^30]", V);
+  if (K < 1 || K > kMaxK) return fail(KDKL_ERR_SHAPE, "K=%d outside [1, %d]", K, kMaxK);
+  if (K > V) return fail(KDKL_ERR_SHAPE, "K=%d larger than V=%d", K, V);
+  if (!std::isfinite(tau) || !(tau > 0.f)) return fail(KDKL_ERR_SHAPE, "tau must be finite and > 0");
+  return KDKL_OK;
+}
+
+struct Common {
+  const void* hidden;
+  const void* W;
+  const int32_t* idx;
+  const float* logit;
+  const uint8_t* mask;
+  int64_t N;
+  int32_t d, V, K;
+  float tau;
+  void* ws;
+  size_t ws_bytes;
+};
+
+kdkl_status check_common(const Common& c, int64_t chunk_tokens, WsLayout& L) {
+  kdkl_status st = check_shapes(c.N, c.d, c.V, c.K, c.tau);
+  if (st != KDKL_OK) return st;
+  if (!c.hidden || !c.W || !c.idx || !c.logit || !c.mask || !c.ws)
+    return fail(KDKL_ERR_NULL, "hidden, W, topk_idx, topk_logit, mask and workspace must be non-NULL");
+  if (!aligned(c.hidden, 16) || !aligned(c.W, 16)) return fail(KDKL_ERR_ALIGN, "hidden and W must be 16-byte aligned");
+  if (!aligned(c.idx, 4) || !aligned(c.logit, 4)) return fail(KDKL_ERR_ALIGN, "topk_idx and topk_logit must be 4-byte aligned");
+  if (!aligned(c.ws, 256)) return fail(KDKL_ERR_ALIGN, "workspace must be 256-byte aligned");
+  if (chunk_tokens < 0) return fail(KDKL_ERR_SHAPE, "chunk_tokens must be >= 0");
+  L = make_layout(c.N, c.d, c.V, c.K, chunk_tokens);
+  if (c.ws_bytes < L.total)
+    return fail(KDKL_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", c.ws_bytes, L.total);
+  return KDKL_OK;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+kdkl_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(KDKL_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// ---------------------------------------------------------------- timing
+enum TimedKind { kTPrepass = 0, kTFwd, kTMerge, kTGrad, kTDh, kTDw, kTKinds };
+const char* const kTimedNames[kTKinds] = {"prepass", "fwd_lse_gemm", "merge", "bwd_grad_gemm", "bwd_dhidden_gemm",
+                                          "bwd_dw_gemm"};
+struct TimingRec {
+  int kind;
+  cudaEvent_t a, b;
+};
+std::mutex g_tmu;
+bool g_timing = false;
+std::vector<TimingRec> g_pending;
+uint64_t g_launches[kTKinds] = {0};
+double g_ms[kTKinds] = {0};
+
+template <class F>
+cudaError_t timed(int kind, cudaStream_t s, F&& launch) {
+  bool on;
+  {
+    std::lock_guard<std::mutex> lk(g_tmu);
+    on = g_timing;
+  }
+  if (!on) return launch();
+  cudaEvent_t a = nullptr, b = nullptr;
+  if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess) return cudaGetLastError();
+  cudaEventRecord(a, s);
+  const cudaError_t e = launch();
+  cudaEventRecord(b, s);
+  std::lock_guard<std::mutex> lk(g_tmu);
+  g_pending.push_back({kind, a, b});
+  return e;
+}
+
+// Prepass shared by forward and backward (the backward keeps no state from the forward).
+kdkl_status run_prepass(const Common& c, const WsLayout& L, cudaStream_t s) {
+  uint32_t* header = at<uint32_t>(c.ws, L.header);
+  cudaError_t e = cudaMemsetAsync(header, 0, 256, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  e = timed(kTPrepass, s, [&] {
+    return launch_prepass(c.idx, c.logit, c.mask, c.N, c.V, c.K, c.tau, at<int>(c.ws, L.sidx),
+                          at<float>(c.ws, L.sprob), at<float>(c.ws, L.negent), at<uint8_t>(c.ws, L.rowmask), L.Kp,
+                          header, s);
+  });
+  if (e != cudaSuccess) return cuda_fail(e, "prepass launch");
+  return KDKL_OK;
+}
+
+EpiParams base_params(const Common& c, const WsLayout& L) {
+  EpiParams ep;
+  std::memset(&ep, 0, sizeof(ep));
+  ep.sidx = at<int>(c.ws, L.sidx);
+  ep.sprob = at<float>(c.ws, L.sprob);
+  ep.Kp = L.Kp;
+  ep.rowmask = at<uint8_t>(c.ws, L.rowmask);
+  ep.n_valid = at<uint32_t>(c.ws, L.header) + 1;
+  ep.flags = at<uint32_t>(c.ws, L.header);
+  return ep;
+}
+
+}  // namespace
+
+WsLayout make_layout(int64_t N, int32_t d, int32_t V, int32_t K, int64_t chunk_tokens) {
+  (void)d;
+  WsLayout L;
+  L.Kp = list_pitch(K);
+  const int64_t rb = (N + kBM - 1) / kBM;
+  L.units_cap = rb * 8 + 4096;
+  int64_t chunk = chunk_tokens > 0 ? chunk_tokens : kDefaultChunk;
+  chunk = (chunk + kBM - 1) / kBM * kBM;
+  const int64_t n_up = (N + kBM - 1) / kBM * kBM;
+  if (chunk > n_up) chunk = n_up;
+  if (chunk < kBM) chunk = kBM;
+  L.chunk = chunk;
+  L.Vp = (static_cast<int64_t>(V) + 63) / 64 * 64;
+  size_t off = 0;
+  L.header = off;
+  off += 256;
+  L.sidx = off;
+  off = align_up(off + static_cast<size_t>(N) * L.Kp * 4, 256);
+  L.sprob = off;
+  off = align_up(off + static_cast<size_t>(N) * L.Kp * 4, 256);
+  L.negent = off;
+  off = align_up(off + static_cast<size_t>(N) * 4, 256);
+  L.rowmask = off;
+  off = align_up(off + static_cast<size_t>(N), 256);
+  L.partial = off;
+  off = align_up(off + static_cast<size_t>(L.units_cap) * kBM * 3 * 4, 256);
+  L.blocksum = off;
+  off = align_up(off + static_cast<size_t>((N + 255) / 256 + 1) * 8, 256);
+  L.gbuf = off;
+  off = align_up(off + static_cast<size_t>(L.chunk) * L.Vp * 2, 256);
+  L.total = off;
+  return L;
+}
+
+}  // namespace kdkl
+
+using namespace kdkl;
+
+extern "C" {
+
+size_t kdkl_workspace_bytes(int64_t N, int32_t d, int32_t V, int32_t K, int64_t chunk_tokens) {
+  if (check_shapes(N, d, V, K, 1.0f) != KDKL_OK || chunk_tokens < 0) return 0;
+  return make_layout(N, d, V, K, chunk_tokens).total;
+}
+
+const char* kdkl_status_string(kdkl_status s) {
+  switch (s) {
+    case KDKL_OK: return "KDKL_OK";
+    case KDKL_ERR_NULL: return "KDKL_ERR_NULL";
+    case KDKL_ERR_SHAPE: return "KDKL_ERR_SHAPE";
+    case KDKL_ERR_ALIGN: return "KDKL_ERR_ALIGN";
+    case KDKL_ERR_UNSUPPORTED: return "KDKL_ERR_UNSUPPORTED";
+    case KDKL_ERR_WORKSPACE: return "KDKL_ERR_WORKSPACE";
+    case KDKL_ERR_CUDA: return "KDKL_ERR_CUDA";
+  }
+  return "KDKL_ERR_UNKNOWN";
+}
+
+const char* kdkl_last_error(void) { return g_last_error; }
+
+kdkl_status kdkl_forward(const void* hidden, const void* W, const int32_t* topk_idx, const float* topk_logit,
+                         const uint8_t* mask, int64_t N, int32_t d, int32_t V, int32_t K, float tau, float* loss,
+                         float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  const Common c{hidden, W, topk_idx, topk_logit, mask, N, d, V, K, tau, workspace, workspace_bytes};
+  WsLayout L;
+  kdkl_status st = check_common(c, 0, L);
+  if (st != KDKL_OK) return st;
+  if (!loss || !lse) return fail(KDKL_ERR_NULL, "loss and lse must be non-NULL");
+  if (!aligned(loss, 4) || !aligned(lse, 4)) return fail(KDKL_ERR_ALIGN, "loss and lse must be 4-byte aligned");
+  Device dv;
+  if ((st = current_device(dv)) != KDKL_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (N == 0) {
+    if ((e = cudaMemsetAsync(workspace, 0, 256, s)) != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+    if ((e = cudaMemsetAsync(loss, 0, sizeof(float), s)) != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+    return ok();
+  }
+  if ((st = run_prepass(c, L, s)) != KDKL_OK) return st;
+
+  const int64_t rb = (N + kBM - 1) / kBM;
+  const int vt = (V + 255) / 256;
+  const int splits = pick_splits(rb, vt, dv.sms, d, L.units_cap);
+  Sched sc;
+  sc.units = static_cast<int>(rb * splits);
+  sc.splits = splits;
+  sc.n_tiles = vt;
+  sc.k_blocks = (d + kBK - 1) / kBK;
+  sc.row_stream = 1;
+  CUtensorMap tmA, tmB;
+  if (!make_map(&tmA, hidden, d, N, d, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tmB, W, d, V, d, kBK, 256, CU_TENSOR_MAP_SWIZZLE_128B))
+    return fail(KDKL_ERR_CUDA, "cuTensorMapEncodeTiled failed (hidden/W)");
+  EpiParams ep = base_params(c, L);
+  ep.M = static_cast<int>(N);
+  ep.Ncols = V;
+  ep.row_offset = 0;
+  float* part = at<float>(workspace, L.partial);
+  const size_t plane = static_cast<size_t>(L.units_cap) * kBM;
+  ep.part_m = part;
+  ep.part_s = part + plane;
+  ep.part_a = part + 2 * plane;
+  const int grid = sc.units < dv.sms ? sc.units : dv.sms;
+  if ((e = timed(kTFwd, s, [&] { return launch_gemm(kEpiLse, 256, tmA, tmB, tmA, sc, ep, grid, s); })) !=
+      cudaSuccess)
+    return cuda_fail(e, "forward GEMM launch");
+  uint32_t* header = at<uint32_t>(workspace, L.header);
+  if ((e = timed(kTMerge, s, [&] {
+         return launch_merge(ep.part_m, ep.part_s, ep.part_a, splits, at<float>(workspace, L.negent),
+                             at<uint8_t>(workspace, L.rowmask), N, lse, loss, at<double>(workspace, L.blocksum),
+                             header, s);
+       })) != cudaSuccess)
+    return cuda_fail(e, "merge launch");
+  return ok();
+}
+
+kdkl_status kdkl_backward(const void* hidden, const void* W, const int32_t* topk_idx, const float* topk_logit,
+                          const uint8_t* mask, int64_t N, int32_t d, int32_t V, int32_t K, float tau, const float* lse,
+                          const float* grad_loss, void* dHidden, float* dW, int64_t chunk_tokens, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  const Common c{hidden, W, topk_idx, topk_logit, mask, N, d, V, K, tau, workspace, workspace_bytes};
+  WsLayout L;
+  kdkl_status st = check_common(c, chunk_tokens, L);
+  if (st != KDKL_OK) return st;
+  if (!lse || !dHidden || !dW) return fail(KDKL_ERR_NULL, "lse, dHidden and dW must be non-NULL");
+  if (!aligned(lse, 4) || (grad_loss && !aligned(grad_loss, 4)))
+    return fail(KDKL_ERR_ALIGN, "lse and grad_loss must be 4-byte aligned");
+  if (!aligned(dHidden, 16) || !aligned(dW, 16)) return fail(KDKL_ERR_ALIGN, "dHidden and dW must be 16-byte aligned");
+  Device dv;
+  if ((st = current_device(dv)) != KDKL_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (N == 0) {
+    if ((e = cudaMemsetAsync(workspace, 0, 256, s)) != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+    if ((e = cudaMemsetAsync(dW, 0, static_cast<size_t>(V) * d * sizeof(float), s)) != cudaSuccess)
+      return cuda_fail(e, "cudaMemsetAsync");
+    return ok();
+  }
+  if ((st = run_prepass(c, L, s)) != KDKL_OK) return st;
+
+  uint16_t* gbuf = at<uint16_t>(workspace, L.gbuf);
+  CUtensorMap tmW_k;  // W as K-major B of the logit recompute
+  CUtensorMap tmW_mn; // W as MN-major B of dHidden = G W
+  if (!make_map(&tmW_k, W, d, V, d, kBK, 256, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tmW_mn, W, d, V, d, 64, kBK, CU_TENSOR_MAP_SWIZZLE_128B))
+    return fail(KDKL_ERR_CUDA, "cuTensorMapEncodeTiled failed (W)");
+  const int vt = (V + 255) / 256;
+  const int bn = pick_bn(d);
+  const int nt = (d + bn - 1) / bn;
+  EpiParams ep0 = base_params(c, L);
+  ep0.lse = lse;
+  ep0.grad_loss = grad_loss;
+
+  for (int64_t c0 = 0; c0 < N; c0 += L.chunk) {
+    const int64_t nc = (N - c0) < L.chunk ? (N - c0) : L.chunk;
+    const void* hc = static_cast<const uint8_t*>(hidden) + static_cast<size_t>(c0) * d * 2;
+    CUtensorMap tmH_k, tmH_mn, tmG_store, tmG_k, tmG_mn;
+    if (!make_map(&tmH_k, hc, d, nc, d, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tmH_mn, hc, d, nc, d, 64, kBK, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tmG_store, gbuf, V, nc, L.Vp, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_map(&tmG_k, gbuf, V, nc, L.Vp, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tmG_mn, gbuf, V, nc, L.Vp, 64, kBK, CU_TENSOR_MAP_SWIZZLE_128B))
+      return fail(KDKL_ERR_CUDA, "cuTensorMapEncodeTiled failed (chunk maps)");
+    const int64_t rbc = (nc + kBM - 1) / kBM;
+
+    // (1) recompute the chunk's logits and form G (bf16) in the chunk buffer
+    {
+      const int splits = pick_splits(rbc, vt, dv.sms, d, L.units_cap);
+      Sched sc{static_cast<int>(rbc * splits), splits, vt, (d + kBK - 1) / kBK, 1};
+      EpiParams ep = ep0;
+      ep.M = static_cast<int>(nc);
+      ep.Ncols = V;
+      ep.row_offset = c0;
+      const int grid = sc.units < dv.sms ? sc.units : dv.sms;
+      if ((e = timed(kTGrad, s, [&] { return launch_gemm(kEpiGrad, 256, tmH_k, tmW_k, tmG_store, sc, ep, grid, s); })) !=
+          cudaSuccess)
+        return cuda_fail(e, "gradient GEMM launch");
+    }
+    // (2) dHidden rows of the chunk = G W
+    {
+      Sched sc{static_cast<int>(rbc * nt), 1, nt, static_cast<int>((V + kBK - 1) / kBK), 0};
+      EpiParams ep = ep0;
+      ep.M = static_cast<int>(nc);
+      ep.Ncols = d;
+      ep.row_offset = c0;
+      ep.dH = static_cast<uint16_t*>(dHidden);
+      ep.ldo = d;
+      const int grid = sc.units < dv.sms ? sc.units : dv.sms;
+      if ((e = timed(kTDh, s, [&] { return launch_gemm(kEpiStoreBf16, bn, tmG_k, tmW_mn, tmG_k, sc, ep, grid, s); })) !=
+          cudaSuccess)
+        return cuda_fail(e, "dHidden GEMM launch");
+    }
+    // (3) dW (+)= G^T hidden_chunk, in chunk order (first chunk overwrites)
+    {
+      const int64_t vb = (V + kBM - 1) / kBM;
+      Sched sc{static_cast<int>(vb * nt), 1, nt, static_cast<int>((nc + kBK - 1) / kBK), 0};
+      EpiParams ep = ep0;
+      ep.M = V;
+      ep.Ncols = d;
+      ep.row_offset = 0;
+      ep.dW = dW;
+      ep.ldo = d;
+      ep.accumulate = c0 > 0 ? 1 : 0;
+      const int grid = sc.units < dv.sms ? sc.units : dv.sms;
+      if ((e = timed(kTDw, s, [&] { return launch_gemm(kEpiRmwF32, bn, tmG_mn, tmH_mn, tmG_mn, sc, ep, grid, s); })) !=
+          cudaSuccess)
+        return cuda_fail(e, "dW GEMM launch");
+    }
+  }
+  return ok();
+}
+
+kdkl_status kdkl_timing_enable(int enable) {
+  std::lock_guard<std::mutex> lk(g_tmu);
+  g_timing = enable != 0;
+  return ok();
+}
+
+int kdkl_timing_read(kdkl_kernel_time* out, int max_entries, int reset) {
+  std::vector<TimingRec> pend;
+  {
+    std::lock_guard<std::mutex> lk(g_tmu);
+    pend.swap(g_pending);
+  }
+  for (const TimingRec& r : pend) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.b) == cudaSuccess && cudaEventElapsedTime(&ms, r.a, r.b) == cudaSuccess) {
+      std::lock_guard<std::mutex> lk(g_tmu);
+      g_launches[r.kind] += 1;
+      g_ms[r.kind] += ms;
+    }
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  std::lock_guard<std::mutex> lk(g_tmu);
+  for (int k = 0; k < kTKinds && k < max_entries && out; ++k) {
+    out[k].name = kTimedNames[k];
+    out[k].launches = g_launches[k];
+    out[k].total_ms = g_ms[k];
+  }
+  if (reset) {
+    for (int k = 0; k < kTKinds; ++k) {
+      g_launches[k] = 0;
+      g_ms[k] = 0;
+    }
+  }
+  return kTKinds;
+}
+
+kdkl_status kdkl_read_device_flags(const void* workspace, void* stream, uint32_t* flags_out) {
+  if (!workspace || !flags_out) return fail(KDKL_ERR_NULL, "workspace and flags_out must be non-NULL");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(flags_out, workspace, sizeof(uint32_t), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device flag word");
+  return ok();
+}
+
+}  // extern "C"

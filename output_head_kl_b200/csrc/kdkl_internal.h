@@ -1,0 +1,103 @@
+// Internal declarations shared by the host API and the kernels (not installed).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace kdkl {
+
+constexpr int kBM = 128;        // rows of one MMA tile (TMEM lanes)
+constexpr int kBK = 64;         // K elements per pipeline stage (one 128-byte swizzle row of bf16)
+constexpr int kMaxK = 256;      // cached entries per row
+constexpr int kSentinel = 0x7FFFFFFF;  // pads each row's sorted index list
+
+// Row-pitch (in int32/f32 elements) of the per-row sorted teacher list:
+// at least one sentinel after the K entries, rounded to 4.
+inline int list_pitch(int K) { return ((K + 1) + 3) & ~3; }
+
+// Workspace layout (all offsets 256-byte aligned).  Header words:
+//   [0] device flag word (KDKL_DEV_* bits)
+//   [1] N_valid (count of rows that enter the loss)
+//   [2] ticket of the loss reduction
+struct WsLayout {
+  size_t header = 0;       // 256 bytes
+  size_t sidx = 0;         // [N, Kp] int32 sorted unique indices (sentinel padded)
+  size_t sprob = 0;        // [N, Kp] f32 teacher probabilities aligned with sidx
+  size_t negent = 0;       // [N] f32 sum_v P log P of the teacher row
+  size_t rowmask = 0;      // [N] uint8 effective mask (mask and row usable)
+  size_t partial = 0;      // [units_cap * 128] x 3 f32 (running max, sum-exp, gathered logit)
+  size_t blocksum = 0;     // [ceil(N / 256)] f64 loss partial sums
+  size_t gbuf = 0;         // [chunk, Vp] bf16 chunk buffer of the logit gradient
+  size_t total = 0;
+  int Kp = 0;
+  int64_t units_cap = 0;
+  int64_t chunk = 0;
+  int64_t Vp = 0;
+};
+
+WsLayout make_layout(int64_t N, int32_t d, int32_t V, int32_t K, int64_t chunk_tokens);
+
+// Work decomposition shared by every role of a GEMM kernel.
+//   row-stream mode: unit u -> row block u / splits, vocabulary tiles
+//     [(j * n_tiles) / splits, ((j + 1) * n_tiles) / splits) with j = u % splits.
+//   tile mode: unit u -> row block u / n_tiles, the single tile u % n_tiles.
+struct Sched {
+  int units;
+  int splits;
+  int n_tiles;
+  int k_blocks;
+  int row_stream;
+};
+
+// Parameters of the fused epilogues (the union of what each kind needs).
+struct EpiParams {
+  // geometry
+  int M;             // valid rows of the A operand (tokens of the chunk, or V for dW)
+  int Ncols;         // valid columns of the output (V for loss tiles, d for gradients)
+  int64_t row_offset;  // global token index of local row 0
+  // teacher lists and per-row data (indexed by global token)
+  const int* sidx;
+  const float* sprob;
+  int Kp;
+  const uint8_t* rowmask;
+  // forward partials
+  float* part_m;
+  float* part_s;
+  float* part_a;
+  // backward scale
+  const float* lse;
+  const float* grad_loss;      // may be null (1.0)
+  const uint32_t* n_valid;     // device counter
+  // gradient outputs
+  uint16_t* dH;        // bf16 bits [N, d]
+  float* dW;           // [V, d]
+  int ldo;             // row pitch (elements) of dH / dW
+  int accumulate;      // dW: add into the existing values
+  uint32_t* flags;     // device flag word
+};
+
+enum EpiKind { kEpiLse = 0, kEpiGrad = 1, kEpiStoreBf16 = 2, kEpiRmwF32 = 3 };
+
+// Launchers (defined in kernels.cu).  Each returns cudaGetLastError() of its launch.
+cudaError_t launch_prepass(const int32_t* topk_idx, const float* topk_logit, const uint8_t* mask, int64_t N,
+                           int32_t V, int32_t K, float tau, int* sidx, float* sprob, float* negent,
+                           uint8_t* rowmask, int Kp, uint32_t* header, cudaStream_t stream);
+
+cudaError_t launch_merge(const float* part_m, const float* part_s, const float* part_a, int splits,
+                         const float* negent, const uint8_t* rowmask, int64_t N, float* lse, float* loss,
+                         double* blocksum, uint32_t* header, cudaStream_t stream);
+
+// GEMM kinds: A/B majorness and epilogue are fixed per kind.
+//   kEpiLse      : A = hidden K-major, B = W K-major, BN = 256, row-stream
+//   kEpiGrad     : A = hidden K-major, B = W K-major, BN = 256, row-stream, TMA store of G
+//   kEpiStoreBf16: A = G K-major,      B = W MN-major, BN from {256, 192, 128}, tile mode
+//   kEpiRmwF32   : A = G MN-major,     B = hidden MN-major, BN from {256, 192, 128}, tile mode
+cudaError_t launch_gemm(int kind, int BN, const CUtensorMap& tmA, const CUtensorMap& tmB,
+                        const CUtensorMap& tmOut, const Sched& sched, const EpiParams& ep, int grid,
+                        cudaStream_t stream);
+
+size_t gemm_smem_bytes(int kind, int BN);
+
+}  // namespace kdkl

@@ -1,0 +1,696 @@
+// Device kernels of the fused chunked KL loss (sm_100a).
+//
+//   prepass : per row, sort the cached (index, logit) pairs by index, merge
+//             repeats, P_T = softmax(logit / tau), teacher sum P log P,
+//             effective mask and N_valid.
+//   gemm    : one warp-specialised tcgen05 kernel template (TMA producer warp,
+//             MMA warp, four epilogue warps reading TMEM) with four fused
+//             epilogues:
+//               kEpiLse       forward: running max / sum-exp / gathered logit per row
+//               kEpiGrad      backward: recomputed logits -> G chunk (bf16, TMA store)
+//               kEpiStoreBf16 dHidden = G W  (fp32 in TMEM, bf16 out)
+//               kEpiRmwF32    dW (+)= G^T hidden (fp32 read-modify-write, no atomics)
+//   merge   : combine the split-vocabulary partials into lse and the loss
+//             (deterministic tree + fixed-order final sum).
+//
+// Method: the fused chunked KL loss of "Efficient Knowledge Distillation for
+// LLMs: Offline Top-K Logits and a Fused Chunked KL Loss" (mind-verse.de
+// article, three-variant list, "Fused chunked KL": the projection is folded
+// into the loss, chunks are discarded, the backward recomputes them; llm-wiki
+// note, section "Fused Chunked KL": softmax, log and KL fused in one kernel).
+#include <cfloat>
+#include <cmath>
+
+#include "kdkl_internal.h"
+#include "sm100.cuh"
+
+namespace kdkl {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ============================================================================
+// prepass: one warp per row
+// ============================================================================
+constexpr int kPreWarps = 8;
+
+__global__ void __launch_bounds__(kPreWarps * 32)
+    prepass_kernel(const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_logit,
+                   const uint8_t* __restrict__ mask, int64_t N, int V, int K, float inv_tau,
+                   int* __restrict__ sidx, float* __restrict__ sprob, float* __restrict__ negent,
+                   uint8_t* __restrict__ rowmask, int Kp, uint32_t* __restrict__ header) {
+  __shared__ int s_key[kPreWarps][kMaxK];
+  __shared__ float s_p[kPreWarps][kMaxK];
+  __shared__ int s_skey[kPreWarps][kMaxK];
+  __shared__ float s_sp[kPreWarps][kMaxK];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int* key = s_key[w];
+  float* pv = s_p[w];
+  int* skey = s_skey[w];
+  float* sp = s_sp[w];
+  uint32_t wflags = 0;
+  uint32_t wvalid = 0;
+  const int64_t warps_total = static_cast<int64_t>(gridDim.x) * kPreWarps;
+  for (int64_t n = static_cast<int64_t>(blockIdx.x) * kPreWarps + w; n < N; n += warps_total) {
+    const int32_t* ip = topk_idx + n * K;
+    const float* lp = topk_logit + n * K;
+    int ki[8];
+    float xi[8];
+    bool keep[8];
+    bool any_keep = false, any_bad = false, any_drop = false;
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int k = lane + 32 * i;
+      ki[i] = 0;
+      xi[i] = -INFINITY;
+      keep[i] = false;
+      if (k < K) {
+        const int id = ip[k];
+        const float x = lp[k] * inv_tau;
+        keep[i] = (id >= 0) && (id < V);
+        ki[i] = id;
+        xi[i] = x;
+        if (!keep[i]) any_drop = true;
+        if (keep[i]) {
+          any_keep = true;
+          if (isnan(x) || x == INFINITY) any_bad = true;
+          else mx = fmaxf(mx, x);
+        }
+      }
+    }
+    any_keep = __any_sync(0xffffffffu, any_keep);
+    any_bad = __any_sync(0xffffffffu, any_bad);
+    any_drop = __any_sync(0xffffffffu, any_drop);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (any_drop) wflags |= 1u;
+    const bool row_ok = any_keep && !any_bad && (mx > -INFINITY);
+    if (any_keep && !row_ok) wflags |= 4u;
+    int* out_i = sidx + n * Kp;
+    float* out_p = sprob + n * Kp;
+    if (!row_ok) {
+      for (int k = lane; k < Kp; k += 32) {
+        out_i[k] = kSentinel;
+        out_p[k] = 0.f;
+      }
+      if (lane == 0) {
+        negent[n] = 0.f;
+        rowmask[n] = 0;
+      }
+      __syncwarp();
+      continue;
+    }
+    // teacher probabilities over the in-range entries
+    float e[8];
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      e[i] = keep[i] ? expf(xi[i] - mx) : 0.f;
+      sum += e[i];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const float inv = 1.f / sum;
+    // sort keys: in-range entries by index, dropped entries after them (key V + k)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int k = lane + 32 * i;
+      if (k < K) {
+        key[k] = keep[i] ? ki[i] : (V + k);
+        pv[k] = e[i] * inv;
+      }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int k = lane + 32 * i;
+      if (k < K) {
+        const int mine = key[k];
+        int rank = 0;
+        for (int j = 0; j < K; ++j) {
+          const int other = key[j];
+          rank += (other < mine) || (other == mine && j < k);
+        }
+        skey[rank] = mine;
+        sp[rank] = pv[k];
+      }
+    }
+    __syncwarp();
+    // merge runs of equal indices, compact, and sum P log P
+    float ent = 0.f;
+    int base = 0;
+    bool dup = false;
+    for (int r0 = 0; r0 < K; r0 += 32) {
+      const int r = r0 + lane;
+      bool start = false;
+      float pm = 0.f;
+      int kk = kSentinel;
+      if (r < K) {
+        kk = skey[r];
+        if (kk < V) {
+          start = (r == 0) || (skey[r - 1] != kk);
+          if (!start) dup = true;
+          if (start) {
+            pm = sp[r];
+            for (int t = r + 1; t < K && skey[t] == kk; ++t) pm += sp[t];
+          }
+        }
+      }
+      const uint32_t ballot = __ballot_sync(0xffffffffu, start);
+      const int pos = base + __popc(ballot & ((1u << lane) - 1u));
+      if (start) {
+        out_i[pos] = kk;
+        out_p[pos] = pm;
+        if (pm > 0.f) ent += pm * logf(pm);
+      }
+      base += __popc(ballot);
+    }
+    for (int k = base + lane; k < Kp; k += 32) {
+      out_i[k] = kSentinel;
+      out_p[k] = 0.f;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ent += __shfl_xor_sync(0xffffffffu, ent, o);
+    if (__any_sync(0xffffffffu, dup)) wflags |= 2u;
+    if (lane == 0) {
+      negent[n] = ent;
+      const uint8_t m = (mask[n] != 0) ? 1 : 0;
+      rowmask[n] = m;
+      wvalid += m;
+    }
+    __syncwarp();
+  }
+  if (lane == 0) {
+    if (wflags) atomicOr(&header[0], wflags);
+    if (wvalid) atomicAdd(&header[1], wvalid);
+  }
+}
+
+cudaError_t launch_prepass(const int32_t* topk_idx, const float* topk_logit, const uint8_t* mask, int64_t N,
+                           int32_t V, int32_t K, float tau, int* sidx, float* sprob, float* negent,
+                           uint8_t* rowmask, int Kp, uint32_t* header, cudaStream_t stream) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t want = (N + kPreWarps - 1) / kPreWarps;
+  const int grid = static_cast<int>(want < static_cast<int64_t>(sms) * 8 ? want : static_cast<int64_t>(sms) * 8);
+  prepass_kernel<<<grid, kPreWarps * 32, 0, stream>>>(topk_idx, topk_logit, mask, N, V, K, 1.0f / tau, sidx,
+                                                       sprob, negent, rowmask, Kp, header);
+  return cudaGetLastError();
+}
+
+// ============================================================================
+// merge: split-vocabulary partials -> lse, per-row KL, loss
+// ============================================================================
+constexpr int kMergeThreads = 256;
+
+__global__ void __launch_bounds__(kMergeThreads)
+    merge_kernel(const float* __restrict__ part_m, const float* __restrict__ part_s,
+                 const float* __restrict__ part_a, int splits, const float* __restrict__ negent,
+                 const uint8_t* __restrict__ rowmask, int64_t N, float* __restrict__ lse,
+                 float* __restrict__ loss, double* __restrict__ blocksum, uint32_t* __restrict__ header) {
+  __shared__ double s_red[kMergeThreads / 32];
+  __shared__ bool s_last;
+  const int64_t n = static_cast<int64_t>(blockIdx.x) * kMergeThreads + threadIdx.x;
+  double kl = 0.0;
+  if (n < N) {
+    const int64_t rb = n >> 7;
+    const int r = static_cast<int>(n & 127);
+    float M = -INFINITY;
+    for (int j = 0; j < splits; ++j) M = fmaxf(M, part_m[(rb * splits + j) * 128 + r]);
+    float s = 0.f, a = 0.f;
+    for (int j = 0; j < splits; ++j) {
+      const int64_t slot = (rb * splits + j) * 128 + r;
+      s += part_s[slot] * expf(part_m[slot] - M);
+      a += part_a[slot];
+    }
+    const float l = M + logf(s);
+    lse[n] = l;
+    if (rowmask[n]) kl = static_cast<double>(negent[n]) - static_cast<double>(a) + static_cast<double>(l);
+  }
+  // block tree reduction (fixed order)
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) kl += __shfl_xor_sync(0xffffffffu, kl, o);
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = kl;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int i = 0; i < kMergeThreads / 32; ++i) t += s_red[i];
+    blocksum[blockIdx.x] = t;
+    __threadfence();
+    const uint32_t ticket = atomicAdd(&header[2], 1u);
+    s_last = (ticket == gridDim.x - 1);
+  }
+  __syncthreads();
+  if (s_last && threadIdx.x == 0) {
+    __threadfence();
+    double t = 0.0;
+    const volatile double* bs = blocksum;
+    for (unsigned i = 0; i < gridDim.x; ++i) t += bs[i];
+    const uint32_t nv = *reinterpret_cast<volatile uint32_t*>(&header[1]);
+    loss[0] = nv > 0 ? static_cast<float>(t / static_cast<double>(nv)) : 0.f;
+    header[2] = 0;
+  }
+}
+
+cudaError_t launch_merge(const float* part_m, const float* part_s, const float* part_a, int splits,
+                         const float* negent, const uint8_t* rowmask, int64_t N, float* lse, float* loss,
+                         double* blocksum, uint32_t* header, cudaStream_t stream) {
+  const int grid = static_cast<int>((N + kMergeThreads - 1) / kMergeThreads);
+  merge_kernel<<<grid, kMergeThreads, 0, stream>>>(part_m, part_s, part_a, splits, negent, rowmask, N, lse, loss,
+                                                   blocksum, header);
+  return cudaGetLastError();
+}
+
+// ============================================================================
+// warp-specialised tcgen05 GEMM with fused epilogues
+// ============================================================================
+template <int KIND, int BN>
+struct GemmCfg {
+  static constexpr bool kAmn = (KIND == kEpiRmwF32);
+  static constexpr bool kBmn = (KIND == kEpiStoreBf16 || KIND == kEpiRmwF32);
+  static constexpr int kABytes = kBM * kBK * 2;
+  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kEpiBytes = (KIND == kEpiGrad) ? 4 * 2 * 2048 : 0;
+  static constexpr int kBarBytes = 256;
+  static constexpr int kSmemLimit = 232448;
+  static constexpr int kStagesFit = (kSmemLimit - 1024 - kEpiBytes - kBarBytes) / kStageBytes;
+  static constexpr int kStages = kStagesFit > 6 ? 6 : kStagesFit;
+  static constexpr int kSmem = 1024 + kStages * kStageBytes + kEpiBytes + kBarBytes;
+  static constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, BN, kAmn, kBmn);
+  static constexpr uint32_t kTmemCols = (2 * BN <= 256) ? 256u : 512u;
+  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
+  static_assert(kStages >= 2, "stages");
+};
+
+__device__ __forceinline__ void unit_range(const Sched& sc, int u, int& mb, int& t0, int& t1) {
+  if (sc.row_stream) {
+    mb = u / sc.splits;
+    const int j = u - mb * sc.splits;
+    t0 = static_cast<int>((static_cast<int64_t>(j) * sc.n_tiles) / sc.splits);
+    t1 = static_cast<int>((static_cast<int64_t>(j + 1) * sc.n_tiles) / sc.splits);
+  } else {
+    mb = u / sc.n_tiles;
+    t0 = u - mb * sc.n_tiles;
+    t1 = t0 + 1;
+  }
+}
+
+// z[off] for a run-time off in [0, 32) without dynamic register indexing.
+__device__ __forceinline__ float pick32(const float (&v)[32], uint32_t off) {
+  float t16[16], t8[8], t4[4], t2[2];
+  const bool b4 = off & 16u, b3 = off & 8u, b2 = off & 4u, b1 = off & 2u, b0 = off & 1u;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) t16[j] = b4 ? v[j + 16] : v[j];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) t8[j] = b3 ? t16[j + 8] : t16[j];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) t4[j] = b2 ? t8[j + 4] : t8[j];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) t2[j] = b1 ? t4[j + 2] : t4[j];
+  return b0 ? t2[1] : t2[0];
+}
+
+// First position of a sorted, sentinel-terminated list whose value is >= v.
+__device__ __forceinline__ int lower_bound_list(const int* __restrict__ lst, int Kp, int v) {
+  int lo = 0, hi = Kp - 1;  // lst[Kp - 1] is always the sentinel
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (lst[mid] < v) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo;
+}
+
+template <int KIND, int BN>
+__global__ void __launch_bounds__(192, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmOut, const Sched sc, const EpiParams ep) {
+  using C = GemmCfg<KIND, BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::kStages * C::kABytes;
+  uint8_t* sEpi = sB + C::kStages * C::kBBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + C::kEpiBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + C::kStages;
+  uint64_t* acc_full = bars + 2 * C::kStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    if (KIND == kEpiGrad) tma_prefetch_desc(&tmOut);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const AbortState ab{abort_flag, ep.flags};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int u = blockIdx.x; u < sc.units; u += gridDim.x) {
+        int mb, t0, t1;
+        unit_range(sc, u, mb, t0, t1);
+        for (int t = t0; t < t1; ++t) {
+          for (int kb = 0; kb < sc.k_blocks; ++kb) {
+            if (!mbar_wait(&empty[stage], phase ^ 1u, ab)) goto producer_done;
+            mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+            uint8_t* a = sA + stage * C::kABytes;
+            uint8_t* b = sB + stage * C::kBBytes;
+            if (C::kAmn) {
+              tma_load_2d(a, &tmA, &full[stage], mb * kBM, kb * kBK);
+              tma_load_2d(a + 8192, &tmA, &full[stage], mb * kBM + 64, kb * kBK);
+            } else {
+              tma_load_2d(a, &tmA, &full[stage], kb * kBK, mb * kBM);
+            }
+            if (C::kBmn) {
+#pragma unroll
+              for (int q = 0; q < BN / 64; ++q) tma_load_2d(b + q * 8192, &tmB, &full[stage], t * BN + q * 64, kb * kBK);
+            } else {
+              tma_load_2d(b, &tmB, &full[stage], kb * kBK, t * BN);
+            }
+            if (++stage == C::kStages) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+      }
+    producer_done:;
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int u = blockIdx.x; u < sc.units; u += gridDim.x) {
+        int mb, t0, t1;
+        unit_range(sc, u, mb, t0, t1);
+        for (int t = t0; t < t1; ++t) {
+          if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, ab)) goto mma_done;
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+          for (int kb = 0; kb < sc.k_blocks; ++kb) {
+            if (!mbar_wait(&full[stage], phase, ab)) goto mma_done;
+            tc_fence_after();
+            const uint32_t a_addr = smem_u32(sA + stage * C::kABytes);
+            const uint32_t b_addr = smem_u32(sB + stage * C::kBBytes);
+#pragma unroll
+            for (int j = 0; j < kBK / 16; ++j) {
+              const uint64_t ad = C::kAmn ? sdesc_sw128(a_addr + j * 2048, 8192, 1024)
+                                          : sdesc_sw128(a_addr + j * 32, 16, 1024);
+              const uint64_t bd = C::kBmn ? sdesc_sw128(b_addr + j * 2048, 8192, 1024)
+                                          : sdesc_sw128(b_addr + j * 32, 16, 1024);
+              umma_bf16(d_tmem, ad, bd, C::kIdesc, (kb | j) != 0 ? 1u : 0u);
+            }
+            umma_commit(&empty[stage]);
+            if (++stage == C::kStages) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+          umma_commit(&acc_full[acc]);
+          acc ^= 1;
+          if (acc == 0) acc_phase ^= 1u;
+        }
+      }
+    mma_done:
+      // every MMA issued above has finished before TMEM is released
+      umma_commit(drain);
+      {
+        const uint32_t a = smem_u32(drain);
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(a, 0)) {
+          if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(ep.flags, kFlagTimeout);
+            break;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue warps
+    const int q = warp & 3;
+    const int row_local = q * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    float g_scale = 0.f;
+    if (KIND == kEpiGrad) {
+      const uint32_t nv = *ep.n_valid;
+      const float g = ep.grad_loss ? *ep.grad_loss : 1.0f;
+      g_scale = nv > 0 ? g / static_cast<float>(nv) : 0.f;
+    }
+    uint8_t* stage_buf = sEpi + (warp - 2) * 4096;
+    int sbuf = 0;
+    for (int u = blockIdx.x; u < sc.units; u += gridDim.x) {
+      int mb, t0, t1;
+      unit_range(sc, u, mb, t0, t1);
+      const int row = mb * kBM + row_local;
+      const bool rv = row < ep.M;
+      const int64_t grow = ep.row_offset + row;
+      // per-row state of the loss epilogues
+      float m_run = -INFINITY, s_run = 0.f, a_run = 0.f;
+      float cn = 0.f, lse_l2 = INFINITY;
+      int kpos = 0, nxt = kSentinel;
+      float nxtp = 0.f;
+      const int* lst = nullptr;
+      const float* lsp = nullptr;
+      if (KIND == kEpiLse || KIND == kEpiGrad) {
+        bool live = rv;
+        if (KIND == kEpiGrad) {
+          cn = (rv && ep.rowmask[grow]) ? g_scale : 0.f;
+          live = (cn != 0.f);
+          if (live) lse_l2 = ep.lse[grow] * kLog2e;
+        }
+        if (live) {
+          lst = ep.sidx + grow * ep.Kp;
+          lsp = ep.sprob + grow * ep.Kp;
+          kpos = lower_bound_list(lst, ep.Kp, t0 * BN);
+          nxt = lst[kpos];
+          nxtp = lsp[kpos];
+        }
+      }
+      for (int t = t0; t < t1; ++t) {
+        if (!mbar_wait(&acc_full[acc], acc_phase, ab)) goto epi_done;
+        tc_fence_after();
+        const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(acc * BN);
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          const int col = t * BN + c * 32;
+          if (col >= ep.Ncols) break;
+          float v[32];
+          tmem_ld32(tbase + c * 32, v);
+          tmem_wait_ld();
+          if (KIND == kEpiLse) {
+            if (col + 32 > ep.Ncols) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (col + j >= ep.Ncols) v[j] = -INFINITY;
+            }
+            float cm = v[0];
+#pragma unroll
+            for (int j = 1; j < 32; ++j) cm = fmaxf(cm, v[j]);
+            const float mn = fmaxf(m_run, cm);
+            const float ms = mn * kLog2e;
+            float acc_s = 0.f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc_s += ex2_approx(fmaf(v[j], kLog2e, -ms));
+            s_run = s_run * ex2_approx((m_run - mn) * kLog2e) + acc_s;
+            m_run = mn;
+            while (nxt < col + 32) {
+              a_run = fmaf(nxtp, pick32(v, static_cast<uint32_t>(nxt - col)), a_run);
+              ++kpos;
+              nxt = lst[kpos];
+              nxtp = lsp[kpos];
+            }
+          } else if (KIND == kEpiGrad) {
+            float g[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) g[j] = cn * ex2_approx(fmaf(v[j], kLog2e, -lse_l2));
+            while (nxt < col + 32) {
+              const uint32_t off = static_cast<uint32_t>(nxt - col);
+              const float cp = cn * nxtp;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) g[j] = (off == static_cast<uint32_t>(j)) ? g[j] - cp : g[j];
+              ++kpos;
+              nxt = lst[kpos];
+              nxtp = lsp[kpos];
+            }
+            // stage 32 rows x 32 columns (bf16, 64-byte swizzle) and store with TMA
+            uint8_t* buf = stage_buf + sbuf * 2048;
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+            const uint32_t sw = static_cast<uint32_t>((lane >> 1) & 3);
+#pragma unroll
+            for (int c16 = 0; c16 < 4; ++c16) {
+              uint4 pk;
+              pk.x = pack_bf16x2(g[c16 * 8 + 0], g[c16 * 8 + 1]);
+              pk.y = pack_bf16x2(g[c16 * 8 + 2], g[c16 * 8 + 3]);
+              pk.z = pack_bf16x2(g[c16 * 8 + 4], g[c16 * 8 + 5]);
+              pk.w = pack_bf16x2(g[c16 * 8 + 6], g[c16 * 8 + 7]);
+              *reinterpret_cast<uint4*>(buf + lane * 64 + ((static_cast<uint32_t>(c16) ^ sw) << 4)) = pk;
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmOut, buf, col, mb * kBM + q * 32);
+              bulk_commit();
+            }
+            sbuf ^= 1;
+          } else if (KIND == kEpiStoreBf16) {
+            if (rv) {
+              uint16_t* dst = ep.dH + grow * ep.ldo + col;
+#pragma unroll
+              for (int g8 = 0; g8 < 4; ++g8) {
+                if (col + g8 * 8 + 8 <= ep.Ncols) {
+                  uint4 pk;
+                  pk.x = pack_bf16x2(v[g8 * 8 + 0], v[g8 * 8 + 1]);
+                  pk.y = pack_bf16x2(v[g8 * 8 + 2], v[g8 * 8 + 3]);
+                  pk.z = pack_bf16x2(v[g8 * 8 + 4], v[g8 * 8 + 5]);
+                  pk.w = pack_bf16x2(v[g8 * 8 + 6], v[g8 * 8 + 7]);
+                  *reinterpret_cast<uint4*>(dst + g8 * 8) = pk;
+                }
+              }
+            }
+          } else {  // kEpiRmwF32
+            if (rv) {
+              float* dst = ep.dW + static_cast<int64_t>(row) * ep.ldo + col;
+#pragma unroll
+              for (int g4 = 0; g4 < 8; ++g4) {
+                if (col + g4 * 4 + 4 <= ep.Ncols) {
+                  float4 o = make_float4(v[g4 * 4 + 0], v[g4 * 4 + 1], v[g4 * 4 + 2], v[g4 * 4 + 3]);
+                  if (ep.accumulate) {
+                    const float4 old = *reinterpret_cast<const float4*>(dst + g4 * 4);
+                    o.x += old.x;
+                    o.y += old.y;
+                    o.z += old.z;
+                    o.w += old.w;
+                  }
+                  *reinterpret_cast<float4*>(dst + g4 * 4) = o;
+                }
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (KIND == kEpiLse && rv) {
+        const int64_t slot = static_cast<int64_t>(u) * kBM + row_local;
+        ep.part_m[slot] = m_run;
+        ep.part_s[slot] = s_run;
+        ep.part_a[slot] = a_run;
+      }
+    }
+  epi_done:
+    if (KIND == kEpiGrad) {
+      if (lane == 0) bulk_wait<0>();
+      __syncwarp();
+    }
+  }
+
+  if (*abort_flag) {
+    // give copies that may still be landing in shared memory time to finish
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 1000000ull) {
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+template <int KIND, int BN>
+static cudaError_t launch_one(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmOut,
+                              const Sched& sc, const EpiParams& ep, int grid, cudaStream_t stream) {
+  using C = GemmCfg<KIND, BN>;
+  static bool configured = false;
+  if (!configured) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(gemm_kernel<KIND, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  gemm_kernel<KIND, BN><<<grid, 192, C::kSmem, stream>>>(tmA, tmB, tmOut, sc, ep);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(int kind, int BN, const CUtensorMap& tmA, const CUtensorMap& tmB,
+                        const CUtensorMap& tmOut, const Sched& sc, const EpiParams& ep, int grid,
+                        cudaStream_t stream) {
+  switch (kind) {
+    case kEpiLse:
+      return launch_one<kEpiLse, 256>(tmA, tmB, tmOut, sc, ep, grid, stream);
+    case kEpiGrad:
+      return launch_one<kEpiGrad, 256>(tmA, tmB, tmOut, sc, ep, grid, stream);
+    case kEpiStoreBf16:
+      if (BN == 256) return launch_one<kEpiStoreBf16, 256>(tmA, tmB, tmOut, sc, ep, grid, stream);
+      if (BN == 192) return launch_one<kEpiStoreBf16, 192>(tmA, tmB, tmOut, sc, ep, grid, stream);
+      if (BN == 128) return launch_one<kEpiStoreBf16, 128>(tmA, tmB, tmOut, sc, ep, grid, stream);
+      break;
+    case kEpiRmwF32:
+      if (BN == 256) return launch_one<kEpiRmwF32, 256>(tmA, tmB, tmOut, sc, ep, grid, stream);
+      if (BN == 192) return launch_one<kEpiRmwF32, 192>(tmA, tmB, tmOut, sc, ep, grid, stream);
+      if (BN == 128) return launch_one<kEpiRmwF32, 128>(tmA, tmB, tmOut, sc, ep, grid, stream);
+      break;
+    default:
+      break;
+  }
+  return cudaErrorInvalidValue;
+}
+
+size_t gemm_smem_bytes(int kind, int BN) {
+  switch (kind) {
+    case kEpiLse:
+      return GemmCfg<kEpiLse, 256>::kSmem;
+    case kEpiGrad:
+      return GemmCfg<kEpiGrad, 256>::kSmem;
+    case kEpiStoreBf16:
+      return BN == 256 ? GemmCfg<kEpiStoreBf16, 256>::kSmem
+                       : (BN == 192 ? GemmCfg<kEpiStoreBf16, 192>::kSmem : GemmCfg<kEpiStoreBf16, 128>::kSmem);
+    default:
+      return BN == 256 ? GemmCfg<kEpiRmwF32, 256>::kSmem
+                       : (BN == 192 ? GemmCfg<kEpiRmwF32, 192>::kSmem : GemmCfg<kEpiRmwF32, 128>::kSmem);
+  }
+}
+
+}  // namespace kdkl
