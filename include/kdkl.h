@@ -89,7 +89,8 @@ size_t kdkl_workspace_bytes(int64_t N, int32_t d, int32_t V, int32_t K, int64_t 
  *   N >= 0, d % 8 == 0 (d >= 8), 1 <= K <= 256, K <= V, tau finite and > 0
  *   loss        [1] fp32 out (device), 4-byte aligned
  *   lse         [N] fp32 out (device), 4-byte aligned; written for every row, masked ones too
- *   workspace   >= kdkl_workspace_bytes(N, d, V, K, 0) bytes, 256-byte aligned
+ *   workspace   >= kdkl_workspace_bytes(N, d, V, K, c) bytes for any chunk size c (the
+ *               forward does not touch the backward's chunk buffer), 256-byte aligned
  * N = 0 writes loss = 0 and nothing else.
  */
 kdkl_status kdkl_forward(const void* hidden, const void* W, const int32_t* topk_idx,

@@ -160,7 +160,9 @@ struct Common {
   size_t ws_bytes;
 };
 
-kdkl_status check_common(const Common& c, int64_t chunk_tokens, WsLayout& L) {
+// The forward only uses the workspace before the chunk buffer, so any
+// chunk_tokens value gives it enough room; the backward needs all of it.
+kdkl_status check_common(const Common& c, int64_t chunk_tokens, bool need_chunk_buffer, WsLayout& L) {
   kdkl_status st = check_shapes(c.N, c.d, c.V, c.K, c.tau);
   if (st != KDKL_OK) return st;
   if (!c.hidden || !c.W || !c.idx || !c.logit || !c.mask || !c.ws)
@@ -170,8 +172,8 @@ kdkl_status check_common(const Common& c, int64_t chunk_tokens, WsLayout& L) {
   if (!aligned(c.ws, 256)) return fail(KDKL_ERR_ALIGN, "workspace must be 256-byte aligned");
   if (chunk_tokens < 0) return fail(KDKL_ERR_SHAPE, "chunk_tokens must be >= 0");
   L = make_layout(c.N, c.d, c.V, c.K, chunk_tokens);
-  if (c.ws_bytes < L.total)
-    return fail(KDKL_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", c.ws_bytes, L.total);
+  const size_t need = need_chunk_buffer ? L.total : L.gbuf;
+  if (c.ws_bytes < need) return fail(KDKL_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", c.ws_bytes, need);
   return KDKL_OK;
 }
 
@@ -309,7 +311,7 @@ kdkl_status kdkl_forward(const void* hidden, const void* W, const int32_t* topk_
                          float* lse, void* workspace, size_t workspace_bytes, void* stream) {
   const Common c{hidden, W, topk_idx, topk_logit, mask, N, d, V, K, tau, workspace, workspace_bytes};
   WsLayout L;
-  kdkl_status st = check_common(c, 0, L);
+  kdkl_status st = check_common(c, 0, false, L);
   if (st != KDKL_OK) return st;
   if (!loss || !lse) return fail(KDKL_ERR_NULL, "loss and lse must be non-NULL");
   if (!aligned(loss, 4) || !aligned(lse, 4)) return fail(KDKL_ERR_ALIGN, "loss and lse must be 4-byte aligned");
@@ -366,7 +368,7 @@ kdkl_status kdkl_backward(const void* hidden, const void* W, const int32_t* topk
                           size_t workspace_bytes, void* stream) {
   const Common c{hidden, W, topk_idx, topk_logit, mask, N, d, V, K, tau, workspace, workspace_bytes};
   WsLayout L;
-  kdkl_status st = check_common(c, chunk_tokens, L);
+  kdkl_status st = check_common(c, chunk_tokens, true, L);
   if (st != KDKL_OK) return st;
   if (!lse || !dHidden || !dW) return fail(KDKL_ERR_NULL, "lse, dHidden and dW must be non-NULL");
   if (!aligned(lse, 4) || (grad_loss && !aligned(grad_loss, 4)))

@@ -1,0 +1,74 @@
+"""Parity at the full workload sizes, in the launch configuration the bench times.
+
+At these sizes the fp64 oracle cannot materialise every logit row in
+seconds, so it checks what it can compute one row at a time:
+
+* lse and dHidden on a seeded sample of rows (each sampled row's full
+  vocabulary logits and gradient row, by the plain definition);
+* the loss, from the oracle's per-row teacher terms over every row
+  (sum P log P and the gathered logit sum_k P_k z[idx_k], both exact per row)
+  combined with the lse the GPU returns for every row, whose own accuracy the
+  sampled check establishes;
+* for dW, properties that hold at any size: every dW column sums to zero
+  (each G row sums to zero), and <dW, W> = <dH, H> (both equal
+  sum_{n,v} G[n, v] z[n, v]).
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import kl as O
+from tests import gpu_harness as H
+
+pytestmark = [pytest.mark.gpu]
+
+SAMPLE = 96
+
+
+def _gather_term(x, W64, rows_per=512):
+    """a_n = sum_k P_k z[n, idx_k] and sum_k P_k log P_k for every row, exact per row in fp64."""
+    N = x.topk_idx.shape[0]
+    V = W64.shape[0]
+    t = O.teacher_distribution(x.topk_idx, x.topk_logit, V, x.tau)
+    m_eff = O.effective_mask(x.mask, t)
+    P = np.where(t.keep, t.P, 0.0)
+    neg = np.where(P > 0, P * np.log(np.where(P > 0, P, 1.0)), 0.0).sum(1)
+    a = np.zeros(N)
+    Wt = torch.from_numpy(W64)
+    idx = torch.from_numpy(np.clip(x.topk_idx.astype(np.int64), 0, V - 1))
+    Pt = torch.from_numpy(P)
+    for r0 in range(0, N, rows_per):
+        r1 = min(N, r0 + rows_per)
+        Hr = torch.from_numpy(O.bf16_bits_to_f64(x.hidden_bits[r0:r1]))
+        Wg = Wt[idx[r0:r1]]                                   # [R, K, d]
+        z = torch.bmm(Wg, Hr[:, :, None])[:, :, 0]           # [R, K] = z[n, idx_k]
+        a[r0:r1] = (Pt[r0:r1] * z).sum(1).numpy()
+    return a, neg, m_eff
+
+
+@pytest.mark.parametrize("name,N", [("8b", None), ("large_vocab", None), ("sweep", 16384)])
+def test_fullsize_sampled(name, N):
+    w = synth.CONFIGS[name]
+    x = synth.make_inputs(w, N=N)
+    g = H.run_gpu(H.to_device(x))
+    assert g.flags == 0
+    rows = synth.sample_rows(x.topk_idx.shape[0], SAMPLE, seed=77)
+    W64 = O.bf16_bits_to_f64(x.W_bits)
+    r = O.kl_loss(x.hidden_bits, x.W_bits, x.topk_idx, x.topk_logit, x.mask, x.tau, rows=rows, want_dW=False,
+                  W_f64=W64)
+    H.assert_lse(g.lse[rows], r.lse)
+    H.assert_grad(g.dH[rows], r.dH, "dHidden (sampled rows)")
+    # loss: oracle per-row teacher terms over all rows + the GPU's lse
+    a, neg, m_eff = _gather_term(x, W64)
+    ref_loss = float(((neg - a + g.lse) * m_eff).sum() / m_eff.sum())
+    H.assert_loss(g.loss, ref_loss)
+    # dW properties
+    col = g.dW.sum(0)
+    assert np.abs(col).max() <= 1e-3 * np.abs(g.dW).max() * np.sqrt(g.dW.shape[0])
+    Hf = O.bf16_bits_to_f64(x.hidden_bits)
+    lhs = float((g.dW * W64).sum())
+    rhs = float((g.dH * Hf).sum())
+    assert abs(lhs - rhs) <= 1e-2 * max(abs(lhs), abs(rhs), 1e-30)
+    del Hf, W64
+    torch.cuda.empty_cache()

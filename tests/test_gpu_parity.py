@@ -117,16 +117,25 @@ def test_one_hot_teacher_is_cross_entropy():
 
 
 def test_full_teacher_K_equals_V():
-    """K = V = 128 with teacher logits equal to the student's own logits: KL ~ 0."""
+    """K = V = 128 with teacher logits equal to the student's own logits: KL ~ 0, grads ~ 0.
+
+    The true gradient is zero here, so it is compared on an absolute scale: the
+    gradient of the same inputs against a shuffled teacher sets the scale."""
     x = synth.custom_inputs(256, 64, 128, 128, seed=109, w_std=0.3)
     Hf = O.bf16_bits_to_f64(x.hidden_bits)
     Wf = O.bf16_bits_to_f64(x.W_bits)
     z = Hf @ Wf.T
     x.topk_idx[:] = np.arange(128, dtype=np.int32)[None, :]
     x.topk_logit[:] = z.astype(np.float32)
-    g, r = _full_parity(x)
+    g = H.run_gpu(H.to_device(x))
+    r = _oracle(x)
     assert abs(r.loss) < 1e-12
     assert abs(g.loss) < 1e-4
+    H.assert_lse(g.lse, r.lse)
+    shuffled = _oracle(synth.Inputs(x.hidden_bits, x.W_bits, x.topk_idx,
+                                    np.ascontiguousarray(x.topk_logit[:, ::-1]), x.mask, x.tau))
+    assert np.abs(g.dH).max() <= 1e-3 * np.abs(shuffled.dH).max()
+    assert np.abs(g.dW).max() <= 1e-3 * np.abs(shuffled.dW).max()
 
 
 def test_constant_W_column_gives_zero_dH_column():
