@@ -118,6 +118,36 @@ kdkl_status kdkl_backward(const void* hidden, const void* W, const int32_t* topk
                           void* stream);
 
 /*
+ * Forward for callers that cannot allocate device memory.  (The paper has no
+ * counterpart of this entry point; it is an interface addition.)
+ *
+ * Some callers cannot hand kdkl a workspace: a loss hook whose host framework
+ * passes only inputs and outputs, a runtime that plans every device byte up
+ * front and forbids later allocations, or a hot loop that must not call
+ * cudaMalloc because an allocation may synchronise the device.  This entry
+ * point takes the same inputs and outputs as kdkl_forward, and the same
+ * results, but no workspace: its scratch is a 32 MiB array built into the
+ * library, which every GPU that loads the library keeps until the process
+ * exits.  It calls no cudaMalloc, cudaFree or other allocating routine.
+ *   - Sizes whose forward scratch exceeds 32 MiB are rejected with
+ *     KDKL_ERR_UNSUPPORTED before any launch: the scratch takes a fixed 6.3 MB
+ *     plus about 8 * K + 130 bytes per token, so up to about 29,000 tokens
+ *     fit at K = 100.
+ *   - The first call on each device looks up that device's copy of the array
+ *     (cudaGetSymbolAddress) with the device current; make that first call
+ *     before any stream capture.
+ *   - Every call on a device shares the one array and leaves its contents
+ *     behind.  Each call clears what must start at zero, so leftovers do not
+ *     matter, but two calls that overlap on the GPU (other streams, other host
+ *     threads) race on the array and corrupt each other's results.
+ *   - The device flag word lives in that array too, so kdkl_read_device_flags
+ *     cannot read it; use kdkl_forward to see data-error flags.
+ */
+kdkl_status kdkl_forward_noalloc(const void* hidden, const void* W, const int32_t* topk_idx,
+                                 const float* topk_logit, const uint8_t* mask, int64_t N, int32_t d,
+                                 int32_t V, int32_t K, float tau, float* loss, float* lse, void* stream);
+
+/*
  * Reads the device flag word of the most recent forward/backward call that
  * used `workspace` (each call clears it first).  Synchronises `stream`.
  */

@@ -134,6 +134,26 @@ def kdkl_backward(hidden, W, topk_idx, topk_logit, mask, tau, lse, grad_loss, dH
     return st
 
 
+def kdkl_forward_noalloc(hidden, W, topk_idx, topk_logit, mask, tau, loss, lse, *, N=None, d=None, V=None,
+                         K=None, stream=None, check=True) -> int:
+    """Calls kdkl_forward_noalloc: the forward without a caller workspace (built-in 32 MiB scratch)."""
+    L = lib()
+    fn = L.kdkl_forward_noalloc
+    vp = ctypes.c_void_p
+    fn.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                   ctypes.c_float, vp, vp, vp]
+    fn.restype = ctypes.c_int
+    N = hidden.shape[0] if N is None else N
+    d = hidden.shape[1] if d is None else d
+    V = W.shape[0] if V is None else V
+    K = topk_idx.shape[1] if K is None else K
+    st = fn(_ptr(hidden), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask), int(N), int(d), int(V), int(K),
+            float(tau), _ptr(loss), _ptr(lse), _stream(stream))
+    if check:
+        _check(st, "kdkl_forward_noalloc")
+    return st
+
+
 def kdkl_read_device_flags(workspace, stream=None) -> int:
     out = ctypes.c_uint32(0)
     _check(lib().kdkl_read_device_flags(_ptr(workspace), _stream(stream), ctypes.byref(out)),

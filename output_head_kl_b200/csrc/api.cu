@@ -280,6 +280,8 @@ WsLayout make_layout(int64_t N, int32_t d, int32_t V, int32_t K, int64_t chunk_t
   return L;
 }
 
+void set_last_error(const char* msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
+
 }  // namespace kdkl
 
 using namespace kdkl;

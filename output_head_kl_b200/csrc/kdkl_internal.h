@@ -100,4 +100,7 @@ cudaError_t launch_gemm(int kind, int BN, const CUtensorMap& tmA, const CUtensor
 
 size_t gemm_smem_bytes(int kind, int BN);
 
+// Sets the message kdkl_last_error() returns on this host thread.
+void set_last_error(const char* msg);
+
 }  // namespace kdkl
