@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N --steps K --warmup W] [--config 8b|small|tiny|large_vocab|sweep] [--N n]
     python bench.py --impl reference ...      # the CPU oracle on a bounded sample (baseline arm)
+    python bench.py --sweep                   # peak GB and tokens/s vs N (d=4096, V=128256, tau=2)
 
 One step = kdkl_forward + kdkl_backward over one batch of seeded synthetic
 inputs already resident in HBM.  Rank 0 prints one JSON line.  With N > 1
@@ -175,6 +176,22 @@ def run_reference(args, w: synth.Workload, N: int):
     return 0
 
 
+# ----------------------------------------------------------------------------- ranks
+def replica_seed(w: synth.Workload, N: int, rank: int) -> int:
+    """Each rank runs an independent replica on its own seeded batch."""
+    return synth.seed_for(w, N) + 7919 * rank
+
+
+def max_over_ranks(value: float, device, world: int) -> float:
+    """The slowest rank's time (a collective only for timing, never on the data path)."""
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ----------------------------------------------------------------------------- GPU arm
 def main_gpu(args, w: synth.Workload, N: int):
     import torch
@@ -193,7 +210,7 @@ def main_gpu(args, w: synth.Workload, N: int):
 
     K.lib()
     t_gen = time.perf_counter()
-    x = synth.make_inputs(w, N=N, seed=synth.seed_for(w, N) + 7919 * rank)
+    x = synth.make_inputs(w, N=N, seed=replica_seed(w, N, rank))
     t_gen = time.perf_counter() - t_gen
     Nn, d, V, Kc = x.shape
 
@@ -254,10 +271,7 @@ def main_gpu(args, w: synth.Workload, N: int):
     kt = K.kdkl_timing_read(reset=True)
     clocks = sampler.stop() if sampler else None
     ms = e0.elapsed_time(e1) / args.steps
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = max_over_ranks(ms, dev, world)
 
     # end-to-end through the public API with host buffers: per step the batch
     # (hidden, cache, mask) goes host -> device from pinned memory and the
@@ -279,10 +293,7 @@ def main_gpu(args, w: synth.Workload, N: int):
         h_loss.copy_(loss, non_blocking=True)
     t1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([t0.elapsed_time(t1) / e2e_steps], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_ms = float(e2e_ms.item())
+    e2e_ms = max_over_ranks(t0.elapsed_time(t1) / e2e_steps, dev, world)
     h2d = Nn * d * 2 + Nn * Kc * 4 * 2 + Nn
     d2h = 4
 
@@ -356,11 +367,22 @@ def main():
     ap.add_argument("--N", type=int, default=None, help="token count override (sweep points)")
     ap.add_argument("--chunk-tokens", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="long-context sweep (d=4096, V=128256, tau=2): one JSON line per N, single GPU")
     args = ap.parse_args()
     w = synth.CONFIGS[args.config]
     N = args.N if args.N is not None else w.N
     if args.impl == "reference":
         return run_reference(args, w, N)
+    if args.sweep:
+        args.no_cpu_baseline = True
+        for n in synth.SWEEP_N:
+            rc = main_gpu(args, synth.CONFIGS["sweep"], n)
+            if rc:
+                return rc
+            import torch
+            torch.cuda.empty_cache()
+        return 0
     return main_gpu(args, w, N)
 
 

@@ -95,10 +95,11 @@ kdkl_status current_device(Device& dv) {
 }
 
 // Vocabulary splits for a row-stream kernel over `rb` row blocks and `vt`
-// vocabulary tiles: balance the per-CTA tile count over `ctas`, and keep at
-// least enough splits that the hidden rows in flight stay small next to L2.
-int pick_splits(int64_t rb, int vt, int ctas, int d, int64_t units_cap) {
-  const double rows_bytes = 128.0 * d * 2.0;
+// vocabulary tiles: balance the per-group tile count over `ctas` CTA groups
+// (single CTAs or CTA pairs), and keep at least enough splits that the hidden
+// rows in flight stay small next to L2.  `units_cap` bounds rb * splits.
+int pick_splits(int64_t rb, int vt, int ctas, int d, int64_t units_cap, int rows_per_block) {
+  const double rows_bytes = static_cast<double>(rows_per_block) * d * 2.0;
   const double budget = 48.0 * 1024 * 1024;
   int s_min = static_cast<int>(std::ceil(ctas * rows_bytes / budget));
   if (s_min < 1) s_min = 1;
@@ -122,19 +123,40 @@ int pick_splits(int64_t rb, int vt, int ctas, int d, int64_t units_cap) {
   return best;
 }
 
+// Tile width of the dHidden / dW GEMMs (their N dimension is d).  256-wide
+// tiles run as CTA pairs (cta_group::2), which keep the tensor pipe about 15
+// points busier per clock than single-CTA tiles, so they win unless padding d
+// up to a multiple of 256 wastes more than 1/8 of the work; then the
+// narrower single-CTA tile with the least padding is used.
 int pick_bn(int d) {
-  // smallest padded width; ties go to the wider tile
-  const int cands[3] = {256, 192, 128};
-  int best = 256;
-  int64_t best_pad = INT64_MAX;
-  for (int c : cands) {
-    const int64_t pad = static_cast<int64_t>((d + c - 1) / c) * c;
-    if (pad < best_pad) {
-      best_pad = pad;
-      best = c;
-    }
+  const int64_t pad256 = static_cast<int64_t>((d + 255) / 256) * 256;
+  const int64_t pad192 = static_cast<int64_t>((d + 191) / 192) * 192;
+  const int64_t pad128 = static_cast<int64_t>((d + 127) / 128) * 128;
+  const int64_t best_narrow = pad192 < pad128 ? pad192 : pad128;
+  if (pad256 * 8 <= best_narrow * 9) return 256;
+  return pad192 <= pad128 ? 192 : 128;
+}
+
+// Whether a GEMM runs as CTA pairs (256-row tiles, cta_group::2) or single
+// CTAs (128-row tiles).  Pairs need the 256-wide N tile (split 128 + 128).
+struct Pairing {
+  bool pair;
+  int rows;     // rows of one tile / unit
+  int groups;   // CTA groups that run at once (pairs or single CTAs)
+  int b_rows;   // rows of the K-major B box one CTA loads
+  int grid(int64_t units) const {
+    const int64_t g = units < groups ? units : groups;
+    return static_cast<int>(pair ? 2 * g : g);
   }
-  return best;
+};
+
+Pairing pairing(const Device& dv, int bn) {
+  Pairing p;
+  p.pair = (bn == 256) && dv.sms >= 2;
+  p.rows = p.pair ? 2 * kBM : kBM;
+  p.groups = p.pair ? dv.sms / 2 : dv.sms;
+  p.b_rows = p.pair ? bn / 2 : bn;
+  return p;
 }
 
 kdkl_status check_shapes(int64_t N, int32_t d, int32_t V, int32_t K, float tau) {
@@ -328,9 +350,10 @@ kdkl_status kdkl_forward(const void* hidden, const void* W, const int32_t* topk_
   }
   if ((st = run_prepass(c, L, s)) != KDKL_OK) return st;
 
-  const int64_t rb = (N + kBM - 1) / kBM;
+  const Pairing pr = pairing(dv, 256);
+  const int64_t rb = (N + pr.rows - 1) / pr.rows;
   const int vt = (V + 255) / 256;
-  const int splits = pick_splits(rb, vt, dv.sms, d, L.units_cap);
+  const int splits = pick_splits(rb, vt, pr.groups, d, L.units_cap * kBM / pr.rows, pr.rows);
   Sched sc;
   sc.units = static_cast<int>(rb * splits);
   sc.splits = splits;
@@ -339,7 +362,7 @@ kdkl_status kdkl_forward(const void* hidden, const void* W, const int32_t* topk_
   sc.row_stream = 1;
   CUtensorMap tmA, tmB;
   if (!make_map(&tmA, hidden, d, N, d, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&tmB, W, d, V, d, kBK, 256, CU_TENSOR_MAP_SWIZZLE_128B))
+      !make_map(&tmB, W, d, V, d, kBK, pr.b_rows, CU_TENSOR_MAP_SWIZZLE_128B))
     return fail(KDKL_ERR_CUDA, "cuTensorMapEncodeTiled failed (hidden/W)");
   EpiParams ep = base_params(c, L);
   ep.M = static_cast<int>(N);
@@ -350,13 +373,13 @@ kdkl_status kdkl_forward(const void* hidden, const void* W, const int32_t* topk_
   ep.part_m = part;
   ep.part_s = part + plane;
   ep.part_a = part + 2 * plane;
-  const int grid = sc.units < dv.sms ? sc.units : dv.sms;
-  if ((e = timed(kTFwd, s, [&] { return launch_gemm(kEpiLse, 256, tmA, tmB, tmA, sc, ep, grid, s); })) !=
+  const int grid = pr.grid(sc.units);
+  if ((e = timed(kTFwd, s, [&] { return launch_gemm(kEpiLse, 256, pr.pair, tmA, tmB, tmA, sc, ep, grid, s); })) !=
       cudaSuccess)
     return cuda_fail(e, "forward GEMM launch");
   uint32_t* header = at<uint32_t>(workspace, L.header);
   if ((e = timed(kTMerge, s, [&] {
-         return launch_merge(ep.part_m, ep.part_s, ep.part_a, splits, at<float>(workspace, L.negent),
+         return launch_merge(ep.part_m, ep.part_s, ep.part_a, splits, pr.rows, at<float>(workspace, L.negent),
                              at<uint8_t>(workspace, L.rowmask), N, lse, loss, at<double>(workspace, L.blocksum),
                              header, s);
        })) != cudaSuccess)
@@ -389,13 +412,15 @@ kdkl_status kdkl_backward(const void* hidden, const void* W, const int32_t* topk
   if ((st = run_prepass(c, L, s)) != KDKL_OK) return st;
 
   uint16_t* gbuf = at<uint16_t>(workspace, L.gbuf);
+  const Pairing pg = pairing(dv, 256);          // logit recompute (always 256-wide vocabulary tiles)
+  const int bn = pick_bn(d);
+  const Pairing pd = pairing(dv, bn);           // dHidden and dW GEMMs
   CUtensorMap tmW_k;  // W as K-major B of the logit recompute
   CUtensorMap tmW_mn; // W as MN-major B of dHidden = G W
-  if (!make_map(&tmW_k, W, d, V, d, kBK, 256, CU_TENSOR_MAP_SWIZZLE_128B) ||
+  if (!make_map(&tmW_k, W, d, V, d, kBK, pg.b_rows, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map(&tmW_mn, W, d, V, d, 64, kBK, CU_TENSOR_MAP_SWIZZLE_128B))
     return fail(KDKL_ERR_CUDA, "cuTensorMapEncodeTiled failed (W)");
   const int vt = (V + 255) / 256;
-  const int bn = pick_bn(d);
   const int nt = (d + bn - 1) / bn;
   EpiParams ep0 = base_params(c, L);
   ep0.lse = lse;
@@ -411,23 +436,25 @@ kdkl_status kdkl_backward(const void* hidden, const void* W, const int32_t* topk
         !make_map(&tmG_k, gbuf, V, nc, L.Vp, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&tmG_mn, gbuf, V, nc, L.Vp, 64, kBK, CU_TENSOR_MAP_SWIZZLE_128B))
       return fail(KDKL_ERR_CUDA, "cuTensorMapEncodeTiled failed (chunk maps)");
-    const int64_t rbc = (nc + kBM - 1) / kBM;
 
     // (1) recompute the chunk's logits and form G (bf16) in the chunk buffer
     {
-      const int splits = pick_splits(rbc, vt, dv.sms, d, L.units_cap);
+      const int64_t rbc = (nc + pg.rows - 1) / pg.rows;
+      const int splits = pick_splits(rbc, vt, pg.groups, d, L.units_cap * kBM / pg.rows, pg.rows);
       Sched sc{static_cast<int>(rbc * splits), splits, vt, (d + kBK - 1) / kBK, 1};
       EpiParams ep = ep0;
       ep.M = static_cast<int>(nc);
       ep.Ncols = V;
       ep.row_offset = c0;
-      const int grid = sc.units < dv.sms ? sc.units : dv.sms;
-      if ((e = timed(kTGrad, s, [&] { return launch_gemm(kEpiGrad, 256, tmH_k, tmW_k, tmG_store, sc, ep, grid, s); })) !=
-          cudaSuccess)
+      const int grid = pg.grid(sc.units);
+      if ((e = timed(kTGrad, s, [&] {
+             return launch_gemm(kEpiGrad, 256, pg.pair, tmH_k, tmW_k, tmG_store, sc, ep, grid, s);
+           })) != cudaSuccess)
         return cuda_fail(e, "gradient GEMM launch");
     }
     // (2) dHidden rows of the chunk = G W
     {
+      const int64_t rbc = (nc + pd.rows - 1) / pd.rows;
       Sched sc{static_cast<int>(rbc * nt), 1, nt, static_cast<int>((V + kBK - 1) / kBK), 0};
       EpiParams ep = ep0;
       ep.M = static_cast<int>(nc);
@@ -435,14 +462,15 @@ kdkl_status kdkl_backward(const void* hidden, const void* W, const int32_t* topk
       ep.row_offset = c0;
       ep.dH = static_cast<uint16_t*>(dHidden);
       ep.ldo = d;
-      const int grid = sc.units < dv.sms ? sc.units : dv.sms;
-      if ((e = timed(kTDh, s, [&] { return launch_gemm(kEpiStoreBf16, bn, tmG_k, tmW_mn, tmG_k, sc, ep, grid, s); })) !=
-          cudaSuccess)
+      const int grid = pd.grid(sc.units);
+      if ((e = timed(kTDh, s, [&] {
+             return launch_gemm(kEpiStoreBf16, bn, pd.pair, tmG_k, tmW_mn, tmG_k, sc, ep, grid, s);
+           })) != cudaSuccess)
         return cuda_fail(e, "dHidden GEMM launch");
     }
     // (3) dW (+)= G^T hidden_chunk, in chunk order (first chunk overwrites)
     {
-      const int64_t vb = (V + kBM - 1) / kBM;
+      const int64_t vb = (V + pd.rows - 1) / pd.rows;
       Sched sc{static_cast<int>(vb * nt), 1, nt, static_cast<int>((nc + kBK - 1) / kBK), 0};
       EpiParams ep = ep0;
       ep.M = V;
@@ -451,9 +479,10 @@ kdkl_status kdkl_backward(const void* hidden, const void* W, const int32_t* topk
       ep.dW = dW;
       ep.ldo = d;
       ep.accumulate = c0 > 0 ? 1 : 0;
-      const int grid = sc.units < dv.sms ? sc.units : dv.sms;
-      if ((e = timed(kTDw, s, [&] { return launch_gemm(kEpiRmwF32, bn, tmG_mn, tmH_mn, tmG_mn, sc, ep, grid, s); })) !=
-          cudaSuccess)
+      const int grid = pd.grid(sc.units);
+      if ((e = timed(kTDw, s, [&] {
+             return launch_gemm(kEpiRmwF32, bn, pd.pair, tmG_mn, tmH_mn, tmG_mn, sc, ep, grid, s);
+           })) != cudaSuccess)
         return cuda_fail(e, "dW GEMM launch");
     }
   }

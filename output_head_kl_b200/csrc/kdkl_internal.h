@@ -86,19 +86,20 @@ cudaError_t launch_prepass(const int32_t* topk_idx, const float* topk_logit, con
                            uint8_t* rowmask, int Kp, uint32_t* header, cudaStream_t stream);
 
 cudaError_t launch_merge(const float* part_m, const float* part_s, const float* part_a, int splits,
-                         const float* negent, const uint8_t* rowmask, int64_t N, float* lse, float* loss,
-                         double* blocksum, uint32_t* header, cudaStream_t stream);
+                         int rows_per_block, const float* negent, const uint8_t* rowmask, int64_t N, float* lse,
+                         float* loss, double* blocksum, uint32_t* header, cudaStream_t stream);
 
 // GEMM kinds: A/B majorness and epilogue are fixed per kind.
 //   kEpiLse      : A = hidden K-major, B = W K-major, BN = 256, row-stream
 //   kEpiGrad     : A = hidden K-major, B = W K-major, BN = 256, row-stream, TMA store of G
 //   kEpiStoreBf16: A = G K-major,      B = W MN-major, BN from {256, 192, 128}, tile mode
 //   kEpiRmwF32   : A = G MN-major,     B = hidden MN-major, BN from {256, 192, 128}, tile mode
-cudaError_t launch_gemm(int kind, int BN, const CUtensorMap& tmA, const CUtensorMap& tmB,
+// pair = true (BN = 256 only): clusters of two CTAs, 256-row tiles, each CTA
+// loading its 128 rows of A and BN/2 rows of B (the B map's box must be BN/2
+// rows for K-major B); grid must be even.  Units then cover 256 rows.
+cudaError_t launch_gemm(int kind, int BN, bool pair, const CUtensorMap& tmA, const CUtensorMap& tmB,
                         const CUtensorMap& tmOut, const Sched& sched, const EpiParams& ep, int grid,
                         cudaStream_t stream);
-
-size_t gemm_smem_bytes(int kind, int BN);
 
 // Sets the message kdkl_last_error() returns on this host thread.
 void set_last_error(const char* msg);

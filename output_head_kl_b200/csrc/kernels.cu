@@ -206,21 +206,22 @@ constexpr int kMergeThreads = 256;
 
 __global__ void __launch_bounds__(kMergeThreads)
     merge_kernel(const float* __restrict__ part_m, const float* __restrict__ part_s,
-                 const float* __restrict__ part_a, int splits, const float* __restrict__ negent,
-                 const uint8_t* __restrict__ rowmask, int64_t N, float* __restrict__ lse,
+                 const float* __restrict__ part_a, int splits, int rows_per_block,
+                 const float* __restrict__ negent, const uint8_t* __restrict__ rowmask, int64_t N,
+                 float* __restrict__ lse,
                  float* __restrict__ loss, double* __restrict__ blocksum, uint32_t* __restrict__ header) {
   __shared__ double s_red[kMergeThreads / 32];
   __shared__ bool s_last;
   const int64_t n = static_cast<int64_t>(blockIdx.x) * kMergeThreads + threadIdx.x;
   double kl = 0.0;
   if (n < N) {
-    const int64_t rb = n >> 7;
-    const int r = static_cast<int>(n & 127);
+    const int64_t rb = n / rows_per_block;
+    const int r = static_cast<int>(n - rb * rows_per_block);
     float M = -INFINITY;
-    for (int j = 0; j < splits; ++j) M = fmaxf(M, part_m[(rb * splits + j) * 128 + r]);
+    for (int j = 0; j < splits; ++j) M = fmaxf(M, part_m[(rb * splits + j) * rows_per_block + r]);
     float s = 0.f, a = 0.f;
     for (int j = 0; j < splits; ++j) {
-      const int64_t slot = (rb * splits + j) * 128 + r;
+      const int64_t slot = (rb * splits + j) * rows_per_block + r;
       s += part_s[slot] * expf(part_m[slot] - M);
       a += part_a[slot];
     }
@@ -254,32 +255,46 @@ __global__ void __launch_bounds__(kMergeThreads)
 }
 
 cudaError_t launch_merge(const float* part_m, const float* part_s, const float* part_a, int splits,
-                         const float* negent, const uint8_t* rowmask, int64_t N, float* lse, float* loss,
-                         double* blocksum, uint32_t* header, cudaStream_t stream) {
+                         int rows_per_block, const float* negent, const uint8_t* rowmask, int64_t N, float* lse,
+                         float* loss, double* blocksum, uint32_t* header, cudaStream_t stream) {
   const int grid = static_cast<int>((N + kMergeThreads - 1) / kMergeThreads);
-  merge_kernel<<<grid, kMergeThreads, 0, stream>>>(part_m, part_s, part_a, splits, negent, rowmask, N, lse, loss,
-                                                   blocksum, header);
+  merge_kernel<<<grid, kMergeThreads, 0, stream>>>(part_m, part_s, part_a, splits, rows_per_block, negent, rowmask,
+                                                   N, lse, loss, blocksum, header);
   return cudaGetLastError();
 }
 
 // ============================================================================
 // warp-specialised tcgen05 GEMM with fused epilogues
+//
+// PAIR = false: one CTA computes a 128 x BN tile (M = 128 MMAs, cta_group::1).
+// PAIR = true : a cluster of two CTAs computes a 256 x BN tile with M = 256
+//               MMAs issued by the even CTA (cta_group::2).  Each CTA loads
+//               its own 128 rows of A and half (BN/2 rows) of B, so per flop
+//               each SM streams a third less operand data from L2 and reads a
+//               third less from shared memory.  Each CTA's TMEM holds the
+//               accumulator rows of its own 128 rows; both epilogues run in
+//               parallel, one per CTA.
 // ============================================================================
-template <int KIND, int BN>
+template <int KIND, int BN, bool PAIR>
 struct GemmCfg {
   static constexpr bool kAmn = (KIND == kEpiRmwF32);
   static constexpr bool kBmn = (KIND == kEpiStoreBf16 || KIND == kEpiRmwF32);
+  static constexpr int kCtaN = PAIR ? BN / 2 : BN;     // B rows (N) held by this CTA
+  static constexpr int kMmaM = PAIR ? 256 : 128;       // rows of one tile across the pair
   static constexpr int kABytes = kBM * kBK * 2;
-  static constexpr int kBBytes = BN * kBK * 2;
-  static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kEpiBytes = (KIND == kEpiGrad) ? 4 * 2 * 2048 : 0;
+  static constexpr int kBBytes = kCtaN * kBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;               // landing in this CTA
+  static constexpr int kTxBytes = (PAIR ? 2 : 1) * kStageBytes;       // counted on the MMA's barrier
+  static constexpr int kEpiBytes = (KIND == kEpiGrad || KIND == kEpiRmwF32) ? 4 * 4096 : 0;
   static constexpr int kBarBytes = 256;
   static constexpr int kSmemLimit = 232448;
   static constexpr int kStagesFit = (kSmemLimit - 1024 - kEpiBytes - kBarBytes) / kStageBytes;
-  static constexpr int kStages = kStagesFit > 6 ? 6 : kStagesFit;
+  static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
   static constexpr int kSmem = 1024 + kStages * kStageBytes + kEpiBytes + kBarBytes;
-  static constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, BN, kAmn, kBmn);
+  static constexpr uint32_t kIdesc = idesc_bf16_f32(kMmaM, BN, kAmn, kBmn);
   static constexpr uint32_t kTmemCols = (2 * BN <= 256) ? 256u : 512u;
+  static constexpr int kAccEmptyArrivals = PAIR ? 8 : 4;
+  static_assert(kCtaN % 64 == 0 || !kBmn, "MN-major B needs whole 64-column atoms per CTA");
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
   static_assert(kStages >= 2, "stages");
 };
@@ -323,11 +338,11 @@ __device__ __forceinline__ int lower_bound_list(const int* __restrict__ lst, int
   return lo;
 }
 
-template <int KIND, int BN>
+template <int KIND, int BN, bool PAIR>
 __global__ void __launch_bounds__(192, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmOut, const Sched sc, const EpiParams ep) {
-  using C = GemmCfg<KIND, BN>;
+  using C = GemmCfg<KIND, BN, PAIR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -343,6 +358,10 @@ __global__ void __launch_bounds__(192, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;   // 0 = the CTA that issues the MMAs
+  const int group = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int ngroups = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
@@ -350,7 +369,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);
+      mbar_init(&acc_empty[b], C::kAccEmptyArrivals);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -362,11 +381,17 @@ __global__ void __launch_bounds__(192, 1)
     if (KIND == kEpiGrad) tma_prefetch_desc(&tmOut);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::kTmemCols);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(tmem_slot, C::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, C::kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if (PAIR) cluster_sync();   // the even CTA's barriers are initialised before any peer signal
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const AbortState ab{abort_flag, ep.flags};
@@ -376,26 +401,48 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      for (int u = blockIdx.x; u < sc.units; u += gridDim.x) {
+      for (int u = group; u < sc.units; u += ngroups) {
         int mb, t0, t1;
         unit_range(sc, u, mb, t0, t1);
+        const int arow = mb * C::kMmaM + static_cast<int>(rank) * kBM;   // this CTA's A rows
         for (int t = t0; t < t1; ++t) {
+          const int bcol = t * BN + static_cast<int>(rank) * C::kCtaN;  // this CTA's B rows (N)
           for (int kb = 0; kb < sc.k_blocks; ++kb) {
             if (!mbar_wait(&empty[stage], phase ^ 1u, ab)) goto producer_done;
-            mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
             uint8_t* a = sA + stage * C::kABytes;
             uint8_t* b = sB + stage * C::kBBytes;
-            if (C::kAmn) {
-              tma_load_2d(a, &tmA, &full[stage], mb * kBM, kb * kBK);
-              tma_load_2d(a + 8192, &tmA, &full[stage], mb * kBM + 64, kb * kBK);
-            } else {
-              tma_load_2d(a, &tmA, &full[stage], kb * kBK, mb * kBM);
-            }
-            if (C::kBmn) {
+            if (PAIR) {
+              // both CTAs' bytes are counted on the even CTA's barrier
+              const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
+              if (rank == 0) mbar_arrive_expect_tx(&full[stage], C::kTxBytes);
+              if (C::kAmn) {
+                tma_load_2d_pair(a, &tmA, bar0, arow, kb * kBK);
+                tma_load_2d_pair(a + 8192, &tmA, bar0, arow + 64, kb * kBK);
+              } else {
+                tma_load_2d_pair(a, &tmA, bar0, kb * kBK, arow);
+              }
+              if (C::kBmn) {
 #pragma unroll
-              for (int q = 0; q < BN / 64; ++q) tma_load_2d(b + q * 8192, &tmB, &full[stage], t * BN + q * 64, kb * kBK);
+                for (int q = 0; q < C::kCtaN / 64; ++q)
+                  tma_load_2d_pair(b + q * 8192, &tmB, bar0, bcol + q * 64, kb * kBK);
+              } else {
+                tma_load_2d_pair(b, &tmB, bar0, kb * kBK, bcol);
+              }
             } else {
-              tma_load_2d(b, &tmB, &full[stage], kb * kBK, t * BN);
+              mbar_arrive_expect_tx(&full[stage], C::kTxBytes);
+              if (C::kAmn) {
+                tma_load_2d(a, &tmA, &full[stage], arow, kb * kBK);
+                tma_load_2d(a + 8192, &tmA, &full[stage], arow + 64, kb * kBK);
+              } else {
+                tma_load_2d(a, &tmA, &full[stage], kb * kBK, arow);
+              }
+              if (C::kBmn) {
+#pragma unroll
+                for (int q = 0; q < C::kCtaN / 64; ++q)
+                  tma_load_2d(b + q * 8192, &tmB, &full[stage], bcol + q * 64, kb * kBK);
+              } else {
+                tma_load_2d(b, &tmB, &full[stage], kb * kBK, bcol);
+              }
             }
             if (++stage == C::kStages) {
               stage = 0;
@@ -408,13 +455,13 @@ __global__ void __launch_bounds__(192, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------------------ MMA issuer (even CTA only)
+    if (lane == 0 && rank == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      for (int u = blockIdx.x; u < sc.units; u += gridDim.x) {
+      for (int u = group; u < sc.units; u += ngroups) {
         int mb, t0, t1;
         unit_range(sc, u, mb, t0, t1);
         for (int t = t0; t < t1; ++t) {
@@ -432,22 +479,26 @@ __global__ void __launch_bounds__(192, 1)
                                           : sdesc_sw128(a_addr + j * 32, 16, 1024);
               const uint64_t bd = C::kBmn ? sdesc_sw128(b_addr + j * 2048, 8192, 1024)
                                           : sdesc_sw128(b_addr + j * 32, 16, 1024);
-              umma_bf16(d_tmem, ad, bd, C::kIdesc, (kb | j) != 0 ? 1u : 0u);
+              if (PAIR) umma_bf16_pair(d_tmem, ad, bd, C::kIdesc, (kb | j) != 0 ? 1u : 0u);
+              else umma_bf16(d_tmem, ad, bd, C::kIdesc, (kb | j) != 0 ? 1u : 0u);
             }
-            umma_commit(&empty[stage]);
+            if (PAIR) umma_commit_pair(&empty[stage], 0x3);
+            else umma_commit(&empty[stage]);
             if (++stage == C::kStages) {
               stage = 0;
               phase ^= 1u;
             }
           }
-          umma_commit(&acc_full[acc]);
+          if (PAIR) umma_commit_pair(&acc_full[acc], 0x3);
+          else umma_commit(&acc_full[acc]);
           acc ^= 1;
           if (acc == 0) acc_phase ^= 1u;
         }
       }
     mma_done:
-      // every MMA issued above has finished before TMEM is released
-      umma_commit(drain);
+      // every MMA issued above has finished before TMEM or shared memory is released
+      if (PAIR) umma_commit_pair(drain, 0x1);
+      else umma_commit(drain);
       {
         const uint32_t a = smem_u32(drain);
         const uint64_t t0 = globaltimer_ns();
@@ -465,6 +516,7 @@ __global__ void __launch_bounds__(192, 1)
     const int q = warp & 3;
     const int row_local = q * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t acc_empty0 = PAIR ? mapa_shared(smem_u32(&acc_empty[0]), 0) : 0u;
     int acc = 0;
     uint32_t acc_phase = 0;
     float g_scale = 0.f;
@@ -473,12 +525,13 @@ __global__ void __launch_bounds__(192, 1)
       const float g = ep.grad_loss ? *ep.grad_loss : 1.0f;
       g_scale = nv > 0 ? g / static_cast<float>(nv) : 0.f;
     }
-    uint8_t* stage_buf = sEpi + (warp - 2) * 4096;
+    uint8_t* wbuf = sEpi + (warp - 2) * 4096;   // this warp's staging (grad: 2 x 2 KB, dW: 4 KB)
     int sbuf = 0;
-    for (int u = blockIdx.x; u < sc.units; u += gridDim.x) {
+    for (int u = group; u < sc.units; u += ngroups) {
       int mb, t0, t1;
       unit_range(sc, u, mb, t0, t1);
-      const int row = mb * kBM + row_local;
+      const int row0 = mb * C::kMmaM + static_cast<int>(rank) * kBM;   // first row of this CTA
+      const int row = row0 + row_local;
       const bool rv = row < ep.M;
       const int64_t grow = ep.row_offset + row;
       // per-row state of the loss epilogues
@@ -550,7 +603,7 @@ __global__ void __launch_bounds__(192, 1)
               nxtp = lsp[kpos];
             }
             // stage 32 rows x 32 columns (bf16, 64-byte swizzle) and store with TMA
-            uint8_t* buf = stage_buf + sbuf * 2048;
+            uint8_t* buf = wbuf + sbuf * 2048;
             if (lane == 0) bulk_wait_read<1>();
             __syncwarp();
             const uint32_t sw = static_cast<uint32_t>((lane >> 1) & 3);
@@ -566,7 +619,7 @@ __global__ void __launch_bounds__(192, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_2d(&tmOut, buf, col, mb * kBM + q * 32);
+              tma_store_2d(&tmOut, buf, col, row0 + q * 32);
               bulk_commit();
             }
             sbuf ^= 1;
@@ -586,33 +639,47 @@ __global__ void __launch_bounds__(192, 1)
               }
             }
           } else {  // kEpiRmwF32
-            if (rv) {
-              float* dst = ep.dW + static_cast<int64_t>(row) * ep.ldo + col;
+            // Transpose the warp's 32 x 32 fp32 block through shared memory so
+            // that each global access is one full 128-byte row segment.
+            // 16-byte chunk q of row r sits at chunk (q ^ (r & 7)): conflict-free both ways.
+            float* fb = reinterpret_cast<float*>(wbuf);
 #pragma unroll
-              for (int g4 = 0; g4 < 8; ++g4) {
-                if (col + g4 * 4 + 4 <= ep.Ncols) {
-                  float4 o = make_float4(v[g4 * 4 + 0], v[g4 * 4 + 1], v[g4 * 4 + 2], v[g4 * 4 + 3]);
-                  if (ep.accumulate) {
-                    const float4 old = *reinterpret_cast<const float4*>(dst + g4 * 4);
-                    o.x += old.x;
-                    o.y += old.y;
-                    o.z += old.z;
-                    o.w += old.w;
-                  }
-                  *reinterpret_cast<float4*>(dst + g4 * 4) = o;
-                }
-              }
+            for (int q4 = 0; q4 < 8; ++q4)
+              *reinterpret_cast<float4*>(fb + lane * 32 + ((q4 ^ (lane & 7)) << 2)) =
+                  make_float4(v[q4 * 4 + 0], v[q4 * 4 + 1], v[q4 * 4 + 2], v[q4 * 4 + 3]);
+            __syncwarp();
+            const int wrow0 = row0 + q * 32;
+            const bool cv = (col + lane) < ep.Ncols;
+            float r[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              r[i] = fb[i * 32 + ((((lane >> 2) ^ (i & 7))) << 2) + (lane & 3)];
+            __syncwarp();
+            float* base = ep.dW + static_cast<int64_t>(wrow0) * ep.ldo + col + lane;
+            if (ep.accumulate) {
+              float old[32];
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                old[i] = (cv && wrow0 + i < ep.M) ? base[static_cast<int64_t>(i) * ep.ldo] : 0.f;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) r[i] += old[i];
             }
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (cv && wrow0 + i < ep.M) base[static_cast<int64_t>(i) * ep.ldo] = r[i];
           }
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        if (lane == 0) {
+          if (PAIR) mbar_arrive_cluster(acc_empty0 + static_cast<uint32_t>(acc) * 8u);
+          else mbar_arrive(&acc_empty[acc]);
+        }
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
       if (KIND == kEpiLse && rv) {
-        const int64_t slot = static_cast<int64_t>(u) * kBM + row_local;
+        const int64_t slot = static_cast<int64_t>(u) * C::kMmaM + static_cast<int>(rank) * kBM + row_local;
         ep.part_m[slot] = m_run;
         ep.part_s[slot] = s_run;
         ep.part_a[slot] = a_run;
@@ -632,65 +699,77 @@ __global__ void __launch_bounds__(192, 1)
     }
   }
   tc_fence_before();
-  __syncthreads();
+  if (PAIR) cluster_sync();   // the peer's shared memory and TMEM stay alive until the pair is done
+  else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::kTmemCols);
+    if (PAIR) tmem_dealloc_pair(tmem_base, C::kTmemCols);
+    else tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 
-template <int KIND, int BN>
+template <int KIND, int BN, bool PAIR>
 static cudaError_t launch_one(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmOut,
                               const Sched& sc, const EpiParams& ep, int grid, cudaStream_t stream) {
-  using C = GemmCfg<KIND, BN>;
+  using C = GemmCfg<KIND, BN, PAIR>;
   static bool configured = false;
   if (!configured) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(gemm_kernel<KIND, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    const cudaError_t e = cudaFuncSetAttribute(gemm_kernel<KIND, BN, PAIR>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  gemm_kernel<KIND, BN><<<grid, 192, C::kSmem, stream>>>(tmA, tmB, tmOut, sc, ep);
+  if (PAIR) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(192, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemm_kernel<KIND, BN, PAIR>, tmA, tmB, tmOut, sc, ep);
+  }
+  gemm_kernel<KIND, BN, PAIR><<<grid, 192, C::kSmem, stream>>>(tmA, tmB, tmOut, sc, ep);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm(int kind, int BN, const CUtensorMap& tmA, const CUtensorMap& tmB,
+cudaError_t launch_gemm(int kind, int BN, bool pair, const CUtensorMap& tmA, const CUtensorMap& tmB,
                         const CUtensorMap& tmOut, const Sched& sc, const EpiParams& ep, int grid,
                         cudaStream_t stream) {
+  if (pair) {
+    if (BN != 256) return cudaErrorInvalidValue;
+    switch (kind) {
+      case kEpiLse: return launch_one<kEpiLse, 256, true>(tmA, tmB, tmOut, sc, ep, grid, stream);
+      case kEpiGrad: return launch_one<kEpiGrad, 256, true>(tmA, tmB, tmOut, sc, ep, grid, stream);
+      case kEpiStoreBf16: return launch_one<kEpiStoreBf16, 256, true>(tmA, tmB, tmOut, sc, ep, grid, stream);
+      case kEpiRmwF32: return launch_one<kEpiRmwF32, 256, true>(tmA, tmB, tmOut, sc, ep, grid, stream);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (kind) {
     case kEpiLse:
-      return launch_one<kEpiLse, 256>(tmA, tmB, tmOut, sc, ep, grid, stream);
+      return launch_one<kEpiLse, 256, false>(tmA, tmB, tmOut, sc, ep, grid, stream);
     case kEpiGrad:
-      return launch_one<kEpiGrad, 256>(tmA, tmB, tmOut, sc, ep, grid, stream);
+      return launch_one<kEpiGrad, 256, false>(tmA, tmB, tmOut, sc, ep, grid, stream);
     case kEpiStoreBf16:
-      if (BN == 256) return launch_one<kEpiStoreBf16, 256>(tmA, tmB, tmOut, sc, ep, grid, stream);
-      if (BN == 192) return launch_one<kEpiStoreBf16, 192>(tmA, tmB, tmOut, sc, ep, grid, stream);
-      if (BN == 128) return launch_one<kEpiStoreBf16, 128>(tmA, tmB, tmOut, sc, ep, grid, stream);
+      if (BN == 256) return launch_one<kEpiStoreBf16, 256, false>(tmA, tmB, tmOut, sc, ep, grid, stream);
+      if (BN == 192) return launch_one<kEpiStoreBf16, 192, false>(tmA, tmB, tmOut, sc, ep, grid, stream);
+      if (BN == 128) return launch_one<kEpiStoreBf16, 128, false>(tmA, tmB, tmOut, sc, ep, grid, stream);
       break;
     case kEpiRmwF32:
-      if (BN == 256) return launch_one<kEpiRmwF32, 256>(tmA, tmB, tmOut, sc, ep, grid, stream);
-      if (BN == 192) return launch_one<kEpiRmwF32, 192>(tmA, tmB, tmOut, sc, ep, grid, stream);
-      if (BN == 128) return launch_one<kEpiRmwF32, 128>(tmA, tmB, tmOut, sc, ep, grid, stream);
+      if (BN == 256) return launch_one<kEpiRmwF32, 256, false>(tmA, tmB, tmOut, sc, ep, grid, stream);
+      if (BN == 192) return launch_one<kEpiRmwF32, 192, false>(tmA, tmB, tmOut, sc, ep, grid, stream);
+      if (BN == 128) return launch_one<kEpiRmwF32, 128, false>(tmA, tmB, tmOut, sc, ep, grid, stream);
       break;
     default:
       break;
   }
   return cudaErrorInvalidValue;
-}
-
-size_t gemm_smem_bytes(int kind, int BN) {
-  switch (kind) {
-    case kEpiLse:
-      return GemmCfg<kEpiLse, 256>::kSmem;
-    case kEpiGrad:
-      return GemmCfg<kEpiGrad, 256>::kSmem;
-    case kEpiStoreBf16:
-      return BN == 256 ? GemmCfg<kEpiStoreBf16, 256>::kSmem
-                       : (BN == 192 ? GemmCfg<kEpiStoreBf16, 192>::kSmem : GemmCfg<kEpiStoreBf16, 128>::kSmem);
-    default:
-      return BN == 256 ? GemmCfg<kEpiRmwF32, 256>::kSmem
-                       : (BN == 192 ? GemmCfg<kEpiRmwF32, 192>::kSmem : GemmCfg<kEpiRmwF32, 128>::kSmem);
-  }
 }
 
 }  // namespace kdkl
