@@ -123,17 +123,43 @@ def effective_mask(mask: np.ndarray, teacher: Teacher) -> np.ndarray:
     return (np.asarray(mask) != 0) & teacher.row_ok
 
 
+@dataclasses.dataclass(frozen=True)
+class Variant:
+    """Loss-design variant (the pages report loss-design ablations without details:
+    chatpaper.ai abstract, last sentences).  The default is the plain KL.
+
+    P_S = softmax(z / student_tau).  Per valid row the loss is
+        gamma * KL(P_T || P_S) + ce_weight * (-log P_S(label))
+    with gamma = kd_weight * (student_tau^2 if kd_scale_tau_sq else 1) (Hinton's
+    tau^2 factor) and the hard-label term only on rows whose label lies in [0, V).
+    """
+    student_tau: float = 1.0
+    kd_weight: float = 1.0
+    kd_scale_tau_sq: bool = False
+    ce_weight: float = 0.0
+
+    @property
+    def gamma(self) -> float:
+        return self.kd_weight * (self.student_tau ** 2 if self.kd_scale_tau_sq else 1.0)
+
+
+PLAIN = Variant()
+
+
 def kl_loss(hidden_bits, W_bits, topk_idx, topk_logit, mask, tau, *, grad_loss: float = 1.0,
             rows: np.ndarray | None = None, row_chunk: int = 64, want_grads: bool = True,
             want_dW: bool = True, want_G: bool = False, W_f64: np.ndarray | None = None,
-            H_f64: np.ndarray | None = None) -> Result:
+            H_f64: np.ndarray | None = None, variant: Variant = PLAIN,
+            labels: np.ndarray | None = None) -> Result:
     """Loss, per-row lse and (optionally) dHidden / dW by the plain definition.
 
     ``rows`` restricts the per-row work (lse, kl, dH) to a subset; N_valid and the
     loss normaliser always come from every row.  The loss itself is only
     returned when every row was processed (``rows is None``), else it is NaN.
     ``W_f64`` / ``H_f64`` replace the bf16 inputs by arbitrary float64 values
-    (the finite-difference pins perturb them continuously).
+    (the finite-difference pins perturb them continuously).  ``variant`` and
+    ``labels`` select a loss-design variant (see ``Variant``); lse is then the
+    log-sum-exp of z / student_tau and ``kl`` holds each row's combined loss.
     """
     idx = np.asarray(topk_idx, dtype=np.int64)
     N, K = idx.shape
@@ -152,21 +178,35 @@ def kl_loss(hidden_bits, W_bits, topk_idx, topk_logit, mask, tau, *, grad_loss: 
     dW = np.zeros((V, d), dtype=np.float64) if (want_grads and want_dW and all_rows) else None
     G_all = np.zeros((rows.size, V), dtype=np.float64) if want_G else None
 
+    ts = float(variant.student_tau)
+    gamma = variant.gamma
+    beta = float(variant.ce_weight)
+    lab = None if labels is None else np.asarray(labels, dtype=np.int64)
     for c0 in range(0, rows.size, row_chunk):
         sel = rows[c0:c0 + row_chunk]
         H = bf16_bits_to_f64(hidden_bits[sel]) if H_f64 is None else np.asarray(H_f64, np.float64)[sel]
-        z = H @ W.T                                   # [R, V] student logits
+        z = (H @ W.T) / ts                            # [R, V] student logits (softened)
         lse_c = _logsumexp(z)
         logP_S = z - lse_c[:, None]
         P_T = _dense_teacher(idx[sel], teacher.P[sel], teacher.keep[sel], V)
         pos = P_T > 0
         safe = np.where(pos, P_T, 1.0)
-        kl_c = np.where(pos, P_T * (np.log(safe) - logP_S), 0.0).sum(axis=1)
+        kl_c = gamma * np.where(pos, P_T * (np.log(safe) - logP_S), 0.0).sum(axis=1)
+        target = gamma * P_T
+        if beta != 0.0 and lab is not None:
+            ls = lab[sel]
+            has = (ls >= 0) & (ls < V)
+            rr = np.nonzero(has)[0]
+            kl_c = kl_c + beta * np.where(has, -logP_S[np.arange(sel.size), np.clip(ls, 0, V - 1)], 0.0)
+            onehot = np.zeros_like(P_T)
+            onehot[rr, ls[rr]] = 1.0
+            target = target + beta * onehot
         valid = m_eff[sel]
         lse[c0:c0 + sel.size] = lse_c
         kl[c0:c0 + sel.size] = np.where(valid, kl_c, 0.0)
         if want_grads or want_G:
-            G = (scale * valid.astype(np.float64))[:, None] * (np.exp(logP_S) - P_T)
+            wsum = target.sum(axis=1, keepdims=True)       # gamma (+ beta where a label counts)
+            G = (scale / ts * valid.astype(np.float64))[:, None] * (wsum * np.exp(logP_S) - target)
             if want_G:
                 G_all[c0:c0 + sel.size] = G
             if want_grads:
