@@ -148,6 +148,52 @@ kdkl_status kdkl_forward_noalloc(const void* hidden, const void* W, const int32_
                                  int32_t V, int32_t K, float tau, float* loss, float* lse, void* stream);
 
 /*
+ * Options of the extended entry points (kdkl_forward_ex / kdkl_backward_ex).
+ * kdkl_options_init fills the defaults, under which the extended entry points
+ * compute exactly what kdkl_forward / kdkl_backward compute.
+ *
+ * Cache format (the llm-wiki note, section "사전 계산 파이프라인", recommends
+ * 16-bit indices and bf16 values, 4 bytes per cached entry):
+ *   KDKL_CACHE_I32_F32  topk_idx int32, topk_logit fp32 (4-byte aligned)
+ *   KDKL_CACHE_U16_BF16 topk_idx uint16, topk_logit bf16 (2-byte aligned); needs V <= 65536
+ *
+ * Loss-design variants (the paper reports ablations on loss design; these are
+ * the standard knowledge-distillation forms, one shared student softmax):
+ *   P_S = softmax(z / student_tau)
+ *   per valid row: gamma * KL(P_T || P_S) + ce_weight * (-log P_S(label))
+ *   gamma = kd_weight * (student_tau^2 if kd_scale_tau_sq else 1)
+ *   labels[n] outside [0, V) (e.g. -100) add no hard-label term for row n.
+ * The loss is still normalised by N_valid; lse is then the log-sum-exp of
+ * z / student_tau, and kdkl_backward_ex must get the same options as the
+ * forward that produced it.
+ */
+typedef enum { KDKL_CACHE_I32_F32 = 0, KDKL_CACHE_U16_BF16 = 1 } kdkl_cache_format;
+
+typedef struct {
+  int32_t cache_format;     /* kdkl_cache_format */
+  float student_tau;        /* finite, > 0 (default 1) */
+  float kd_weight;          /* finite, >= 0 (default 1) */
+  int32_t kd_scale_tau_sq;  /* nonzero: multiply the KL term by student_tau^2 (default 0) */
+  float ce_weight;          /* finite, >= 0 (default 0: no hard-label term) */
+  const int32_t* labels;    /* [N] int32 device, 4-byte aligned; required when ce_weight > 0 */
+} kdkl_options;
+
+void kdkl_options_init(kdkl_options* options);
+
+/* kdkl_forward with options (NULL = defaults); topk_idx / topk_logit typed by options->cache_format. */
+kdkl_status kdkl_forward_ex(const void* hidden, const void* W, const void* topk_idx, const void* topk_logit,
+                            const uint8_t* mask, int64_t N, int32_t d, int32_t V, int32_t K, float tau,
+                            const kdkl_options* options, float* loss, float* lse, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/* kdkl_backward with options (NULL = defaults); must match the forward's options. */
+kdkl_status kdkl_backward_ex(const void* hidden, const void* W, const void* topk_idx, const void* topk_logit,
+                             const uint8_t* mask, int64_t N, int32_t d, int32_t V, int32_t K, float tau,
+                             const kdkl_options* options, const float* lse, const float* grad_loss,
+                             void* dHidden, float* dW, int64_t chunk_tokens, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/*
  * Reads the device flag word of the most recent forward/backward call that
  * used `workspace` (each call clears it first).  Synchronises `stream`.
  */

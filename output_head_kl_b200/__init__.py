@@ -6,7 +6,8 @@ no fallback: if the library is missing, importing a function that needs it
 raises.
 
 Names mirror the C entry points: ``kdkl_workspace_bytes``, ``kdkl_forward``,
-``kdkl_backward``, ``kdkl_read_device_flags``, ``kdkl_timing_enable``,
+``kdkl_backward``, ``kdkl_forward_ex``, ``kdkl_backward_ex`` (with ``kdkl_options``),
+``kdkl_forward_noalloc``, ``kdkl_read_device_flags``, ``kdkl_timing_enable``,
 ``kdkl_timing_read``, ``kdkl_status_string``, ``kdkl_last_error``.  ``fused_kl_forward_backward`` is a convenience wrapper
 that allocates the outputs and the workspace with torch (the library itself
 never allocates).
@@ -29,6 +30,28 @@ _lib = None
 
 class KernelTime(ctypes.Structure):
     _fields_ = [("name", ctypes.c_char_p), ("launches", ctypes.c_uint64), ("total_ms", ctypes.c_double)]
+
+
+CACHE_I32_F32, CACHE_U16_BF16 = 0, 1
+
+
+class Options(ctypes.Structure):
+    """kdkl_options: cache format and loss-design variant (see include/kdkl.h)."""
+    _fields_ = [("cache_format", ctypes.c_int32), ("student_tau", ctypes.c_float), ("kd_weight", ctypes.c_float),
+                ("kd_scale_tau_sq", ctypes.c_int32), ("ce_weight", ctypes.c_float), ("labels", ctypes.c_void_p)]
+
+
+def kdkl_options(cache_format=CACHE_I32_F32, student_tau=1.0, kd_weight=1.0, kd_scale_tau_sq=False,
+                 ce_weight=0.0, labels=None) -> Options:
+    o = Options()
+    lib().kdkl_options_init(ctypes.byref(o))
+    o.cache_format = int(cache_format)
+    o.student_tau = float(student_tau)
+    o.kd_weight = float(kd_weight)
+    o.kd_scale_tau_sq = 1 if kd_scale_tau_sq else 0
+    o.ce_weight = float(ce_weight)
+    o.labels = _ptr(labels)
+    return o
 
 
 class KDKLError(RuntimeError):
@@ -59,6 +82,14 @@ def lib() -> ctypes.CDLL:
     L.kdkl_status_string.restype = ctypes.c_char_p
     L.kdkl_last_error.argtypes = []
     L.kdkl_last_error.restype = ctypes.c_char_p
+    L.kdkl_options_init.argtypes = [ctypes.POINTER(Options)]
+    L.kdkl_options_init.restype = None
+    L.kdkl_forward_ex.argtypes = [vp, vp, vp, vp, vp, i64, i32, i32, i32, f32, ctypes.POINTER(Options), vp, vp, vp,
+                                  sz, vp]
+    L.kdkl_forward_ex.restype = ctypes.c_int
+    L.kdkl_backward_ex.argtypes = [vp, vp, vp, vp, vp, i64, i32, i32, i32, f32, ctypes.POINTER(Options), vp, vp, vp,
+                                   vp, i64, vp, sz, vp]
+    L.kdkl_backward_ex.restype = ctypes.c_int
     L.kdkl_timing_enable.argtypes = [ctypes.c_int]
     L.kdkl_timing_enable.restype = ctypes.c_int
     L.kdkl_timing_read.argtypes = [ctypes.POINTER(KernelTime), ctypes.c_int, ctypes.c_int]
@@ -131,6 +162,41 @@ def kdkl_backward(hidden, W, topk_idx, topk_logit, mask, tau, lse, grad_loss, dH
                              int(chunk_tokens), _ptr(workspace), int(wsb), _stream(stream))
     if check:
         _check(st, "kdkl_backward")
+    return st
+
+
+def kdkl_forward_ex(hidden, W, topk_idx, topk_logit, mask, tau, loss, lse, workspace, options=None, *, N=None,
+                    d=None, V=None, K=None, workspace_bytes=None, stream=None, check=True) -> int:
+    """Calls kdkl_forward_ex (options: an ``Options`` from ``kdkl_options(...)`` or None)."""
+    N = hidden.shape[0] if N is None else N
+    d = hidden.shape[1] if d is None else d
+    V = W.shape[0] if V is None else V
+    K = topk_idx.shape[1] if K is None else K
+    wsb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    opt = ctypes.byref(options) if options is not None else None
+    st = lib().kdkl_forward_ex(_ptr(hidden), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask), int(N), int(d),
+                               int(V), int(K), float(tau), opt, _ptr(loss), _ptr(lse), _ptr(workspace), int(wsb),
+                               _stream(stream))
+    if check:
+        _check(st, "kdkl_forward_ex")
+    return st
+
+
+def kdkl_backward_ex(hidden, W, topk_idx, topk_logit, mask, tau, lse, grad_loss, dHidden, dW, workspace,
+                     options=None, *, chunk_tokens=0, N=None, d=None, V=None, K=None, workspace_bytes=None,
+                     stream=None, check=True) -> int:
+    """Calls kdkl_backward_ex (same options as the forward)."""
+    N = hidden.shape[0] if N is None else N
+    d = hidden.shape[1] if d is None else d
+    V = W.shape[0] if V is None else V
+    K = topk_idx.shape[1] if K is None else K
+    wsb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    opt = ctypes.byref(options) if options is not None else None
+    st = lib().kdkl_backward_ex(_ptr(hidden), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask), int(N),
+                                int(d), int(V), int(K), float(tau), opt, _ptr(lse), _ptr(grad_loss), _ptr(dHidden),
+                                _ptr(dW), int(chunk_tokens), _ptr(workspace), int(wsb), _stream(stream))
+    if check:
+        _check(st, "kdkl_backward_ex")
     return st
 
 

@@ -172,15 +172,47 @@ kdkl_status check_shapes(int64_t N, int32_t d, int32_t V, int32_t K, float tau) 
 struct Common {
   const void* hidden;
   const void* W;
-  const int32_t* idx;
-  const float* logit;
+  const void* idx;
+  const void* logit;
   const uint8_t* mask;
   int64_t N;
   int32_t d, V, K;
   float tau;
   void* ws;
   size_t ws_bytes;
+  kdkl_options opt;
 };
+
+kdkl_options default_options() {
+  kdkl_options o;
+  std::memset(&o, 0, sizeof(o));
+  o.cache_format = KDKL_CACHE_I32_F32;
+  o.student_tau = 1.0f;
+  o.kd_weight = 1.0f;
+  o.kd_scale_tau_sq = 0;
+  o.ce_weight = 0.0f;
+  o.labels = nullptr;
+  return o;
+}
+
+float kd_gamma(const kdkl_options& o) {
+  return o.kd_weight * (o.kd_scale_tau_sq ? o.student_tau * o.student_tau : 1.0f);
+}
+
+kdkl_status check_options(const Common& c) {
+  const kdkl_options& o = c.opt;
+  if (o.cache_format != KDKL_CACHE_I32_F32 && o.cache_format != KDKL_CACHE_U16_BF16)
+    return fail(KDKL_ERR_UNSUPPORTED, "unknown cache_format %d", o.cache_format);
+  if (o.cache_format == KDKL_CACHE_U16_BF16 && c.V > 65536)
+    return fail(KDKL_ERR_SHAPE, "the 16-bit index cache needs V <= 65536 (V=%d)", c.V);
+  if (!std::isfinite(o.student_tau) || !(o.student_tau > 0.f))
+    return fail(KDKL_ERR_SHAPE, "student_tau must be finite and > 0");
+  if (!std::isfinite(o.kd_weight) || o.kd_weight < 0.f || !std::isfinite(o.ce_weight) || o.ce_weight < 0.f)
+    return fail(KDKL_ERR_SHAPE, "kd_weight and ce_weight must be finite and >= 0");
+  if (o.ce_weight > 0.f && !o.labels) return fail(KDKL_ERR_NULL, "ce_weight > 0 needs labels");
+  if (o.labels && !aligned(o.labels, 4)) return fail(KDKL_ERR_ALIGN, "labels must be 4-byte aligned");
+  return KDKL_OK;
+}
 
 // The forward only uses the workspace before the chunk buffer, so any
 // chunk_tokens value gives it enough room; the backward needs all of it.
@@ -190,7 +222,11 @@ kdkl_status check_common(const Common& c, int64_t chunk_tokens, bool need_chunk_
   if (!c.hidden || !c.W || !c.idx || !c.logit || !c.mask || !c.ws)
     return fail(KDKL_ERR_NULL, "hidden, W, topk_idx, topk_logit, mask and workspace must be non-NULL");
   if (!aligned(c.hidden, 16) || !aligned(c.W, 16)) return fail(KDKL_ERR_ALIGN, "hidden and W must be 16-byte aligned");
-  if (!aligned(c.idx, 4) || !aligned(c.logit, 4)) return fail(KDKL_ERR_ALIGN, "topk_idx and topk_logit must be 4-byte aligned");
+  st = check_options(c);
+  if (st != KDKL_OK) return st;
+  const size_t cache_align = c.opt.cache_format == KDKL_CACHE_U16_BF16 ? 2 : 4;
+  if (!aligned(c.idx, cache_align) || !aligned(c.logit, cache_align))
+    return fail(KDKL_ERR_ALIGN, "topk_idx and topk_logit must be %zu-byte aligned", cache_align);
   if (!aligned(c.ws, 256)) return fail(KDKL_ERR_ALIGN, "workspace must be 256-byte aligned");
   if (chunk_tokens < 0) return fail(KDKL_ERR_SHAPE, "chunk_tokens must be >= 0");
   L = make_layout(c.N, c.d, c.V, c.K, chunk_tokens);
@@ -246,8 +282,9 @@ kdkl_status run_prepass(const Common& c, const WsLayout& L, cudaStream_t s) {
   cudaError_t e = cudaMemsetAsync(header, 0, 256, s);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
   e = timed(kTPrepass, s, [&] {
-    return launch_prepass(c.idx, c.logit, c.mask, c.N, c.V, c.K, c.tau, at<int>(c.ws, L.sidx),
-                          at<float>(c.ws, L.sprob), at<float>(c.ws, L.negent), at<uint8_t>(c.ws, L.rowmask), L.Kp,
+    return launch_prepass(c.opt.cache_format, c.idx, c.logit, c.mask, c.opt.labels, c.N, c.V, c.K, c.tau,
+                          kd_gamma(c.opt), c.opt.ce_weight, at<int>(c.ws, L.sidx), at<float>(c.ws, L.sprob),
+                          at<float>(c.ws, L.negent), at<float>(c.ws, L.wsum), at<uint8_t>(c.ws, L.rowmask), L.Kp,
                           header, s);
   });
   if (e != cudaSuccess) return cuda_fail(e, "prepass launch");
@@ -263,6 +300,9 @@ EpiParams base_params(const Common& c, const WsLayout& L) {
   ep.rowmask = at<uint8_t>(c.ws, L.rowmask);
   ep.n_valid = at<uint32_t>(c.ws, L.header) + 1;
   ep.flags = at<uint32_t>(c.ws, L.header);
+  ep.inv_tau_s = 1.0f / c.opt.student_tau;
+  ep.exp_scale = 1.4426950408889634f / c.opt.student_tau;
+  ep.wsum = at<float>(c.ws, L.wsum);
   return ep;
 }
 
@@ -289,6 +329,8 @@ WsLayout make_layout(int64_t N, int32_t d, int32_t V, int32_t K, int64_t chunk_t
   L.sprob = off;
   off = align_up(off + static_cast<size_t>(N) * L.Kp * 4, 256);
   L.negent = off;
+  off = align_up(off + static_cast<size_t>(N) * 4, 256);
+  L.wsum = off;
   off = align_up(off + static_cast<size_t>(N) * 4, 256);
   L.rowmask = off;
   off = align_up(off + static_cast<size_t>(N), 256);
@@ -330,10 +372,12 @@ const char* kdkl_status_string(kdkl_status s) {
 
 const char* kdkl_last_error(void) { return g_last_error; }
 
-kdkl_status kdkl_forward(const void* hidden, const void* W, const int32_t* topk_idx, const float* topk_logit,
-                         const uint8_t* mask, int64_t N, int32_t d, int32_t V, int32_t K, float tau, float* loss,
-                         float* lse, void* workspace, size_t workspace_bytes, void* stream) {
-  const Common c{hidden, W, topk_idx, topk_logit, mask, N, d, V, K, tau, workspace, workspace_bytes};
+static kdkl_status forward_impl(const void* hidden, const void* W, const void* topk_idx, const void* topk_logit,
+                                const uint8_t* mask, int64_t N, int32_t d, int32_t V, int32_t K, float tau,
+                                const kdkl_options* options, float* loss, float* lse, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  const Common c{hidden,    W,         topk_idx,        topk_logit, mask, N, d, V, K, tau,
+                 workspace, workspace_bytes, options ? *options : default_options()};
   WsLayout L;
   kdkl_status st = check_common(c, 0, false, L);
   if (st != KDKL_OK) return st;
@@ -379,7 +423,8 @@ kdkl_status kdkl_forward(const void* hidden, const void* W, const int32_t* topk_
     return cuda_fail(e, "forward GEMM launch");
   uint32_t* header = at<uint32_t>(workspace, L.header);
   if ((e = timed(kTMerge, s, [&] {
-         return launch_merge(ep.part_m, ep.part_s, ep.part_a, splits, pr.rows, at<float>(workspace, L.negent),
+         return launch_merge(ep.part_m, ep.part_s, ep.part_a, splits, pr.rows, c.opt.student_tau,
+                             at<float>(workspace, L.negent), at<float>(workspace, L.wsum),
                              at<uint8_t>(workspace, L.rowmask), N, lse, loss, at<double>(workspace, L.blocksum),
                              header, s);
        })) != cudaSuccess)
@@ -387,11 +432,28 @@ kdkl_status kdkl_forward(const void* hidden, const void* W, const int32_t* topk_
   return ok();
 }
 
-kdkl_status kdkl_backward(const void* hidden, const void* W, const int32_t* topk_idx, const float* topk_logit,
-                          const uint8_t* mask, int64_t N, int32_t d, int32_t V, int32_t K, float tau, const float* lse,
-                          const float* grad_loss, void* dHidden, float* dW, int64_t chunk_tokens, void* workspace,
-                          size_t workspace_bytes, void* stream) {
-  const Common c{hidden, W, topk_idx, topk_logit, mask, N, d, V, K, tau, workspace, workspace_bytes};
+kdkl_status kdkl_forward(const void* hidden, const void* W, const int32_t* topk_idx, const float* topk_logit,
+                         const uint8_t* mask, int64_t N, int32_t d, int32_t V, int32_t K, float tau, float* loss,
+                         float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  return forward_impl(hidden, W, topk_idx, topk_logit, mask, N, d, V, K, tau, nullptr, loss, lse, workspace,
+                      workspace_bytes, stream);
+}
+
+kdkl_status kdkl_forward_ex(const void* hidden, const void* W, const void* topk_idx, const void* topk_logit,
+                            const uint8_t* mask, int64_t N, int32_t d, int32_t V, int32_t K, float tau,
+                            const kdkl_options* options, float* loss, float* lse, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  return forward_impl(hidden, W, topk_idx, topk_logit, mask, N, d, V, K, tau, options, loss, lse, workspace,
+                      workspace_bytes, stream);
+}
+
+static kdkl_status backward_impl(const void* hidden, const void* W, const void* topk_idx, const void* topk_logit,
+                                 const uint8_t* mask, int64_t N, int32_t d, int32_t V, int32_t K, float tau,
+                                 const kdkl_options* options, const float* lse, const float* grad_loss,
+                                 void* dHidden, float* dW, int64_t chunk_tokens, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  const Common c{hidden,    W,         topk_idx,        topk_logit, mask, N, d, V, K, tau,
+                 workspace, workspace_bytes, options ? *options : default_options()};
   WsLayout L;
   kdkl_status st = check_common(c, chunk_tokens, true, L);
   if (st != KDKL_OK) return st;
@@ -487,6 +549,26 @@ kdkl_status kdkl_backward(const void* hidden, const void* W, const int32_t* topk
     }
   }
   return ok();
+}
+
+kdkl_status kdkl_backward(const void* hidden, const void* W, const int32_t* topk_idx, const float* topk_logit,
+                          const uint8_t* mask, int64_t N, int32_t d, int32_t V, int32_t K, float tau, const float* lse,
+                          const float* grad_loss, void* dHidden, float* dW, int64_t chunk_tokens, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  return backward_impl(hidden, W, topk_idx, topk_logit, mask, N, d, V, K, tau, nullptr, lse, grad_loss, dHidden, dW,
+                       chunk_tokens, workspace, workspace_bytes, stream);
+}
+
+kdkl_status kdkl_backward_ex(const void* hidden, const void* W, const void* topk_idx, const void* topk_logit,
+                             const uint8_t* mask, int64_t N, int32_t d, int32_t V, int32_t K, float tau,
+                             const kdkl_options* options, const float* lse, const float* grad_loss, void* dHidden,
+                             float* dW, int64_t chunk_tokens, void* workspace, size_t workspace_bytes, void* stream) {
+  return backward_impl(hidden, W, topk_idx, topk_logit, mask, N, d, V, K, tau, options, lse, grad_loss, dHidden, dW,
+                       chunk_tokens, workspace, workspace_bytes, stream);
+}
+
+void kdkl_options_init(kdkl_options* options) {
+  if (options) *options = default_options();
 }
 
 kdkl_status kdkl_timing_enable(int enable) {

@@ -13,9 +13,10 @@ constexpr int kBK = 64;         // K elements per pipeline stage (one 128-byte s
 constexpr int kMaxK = 256;      // cached entries per row
 constexpr int kSentinel = 0x7FFFFFFF;  // pads each row's sorted index list
 
-// Row-pitch (in int32/f32 elements) of the per-row sorted teacher list:
-// at least one sentinel after the K entries, rounded to 4.
-inline int list_pitch(int K) { return ((K + 1) + 3) & ~3; }
+// Row-pitch (in int32/f32 elements) of the per-row sorted target list:
+// room for the K cached entries and a hard label, then at least one sentinel,
+// rounded to 4.
+inline int list_pitch(int K) { return ((K + 2) + 3) & ~3; }   // K entries + a hard label + a sentinel
 
 // Workspace layout (all offsets 256-byte aligned).  Header words:
 //   [0] device flag word (KDKL_DEV_* bits)
@@ -25,7 +26,8 @@ struct WsLayout {
   size_t header = 0;       // 256 bytes
   size_t sidx = 0;         // [N, Kp] int32 sorted unique indices (sentinel padded)
   size_t sprob = 0;        // [N, Kp] f32 teacher probabilities aligned with sidx
-  size_t negent = 0;       // [N] f32 sum_v P log P of the teacher row
+  size_t negent = 0;       // [N] f32 gamma * sum_v P_T log P_T of the teacher row
+  size_t wsum = 0;         // [N] f32 total target weight of the row (gamma + beta if it has a label)
   size_t rowmask = 0;      // [N] uint8 effective mask (mask and row usable)
   size_t partial = 0;      // [units_cap * 128] x 3 f32 (running max, sum-exp, gathered logit)
   size_t blocksum = 0;     // [ceil(N / 256)] f64 loss partial sums
@@ -66,6 +68,10 @@ struct EpiParams {
   float* part_m;
   float* part_s;
   float* part_a;
+  // student temperature: exp_scale = log2(e) / tau_s, inv_tau_s = 1 / tau_s
+  float exp_scale;
+  float inv_tau_s;
+  const float* wsum;           // per-row total target weight
   // backward scale
   const float* lse;
   const float* grad_loss;      // may be null (1.0)
@@ -81,13 +87,16 @@ struct EpiParams {
 enum EpiKind { kEpiLse = 0, kEpiGrad = 1, kEpiStoreBf16 = 2, kEpiRmwF32 = 3 };
 
 // Launchers (defined in kernels.cu).  Each returns cudaGetLastError() of its launch.
-cudaError_t launch_prepass(const int32_t* topk_idx, const float* topk_logit, const uint8_t* mask, int64_t N,
-                           int32_t V, int32_t K, float tau, int* sidx, float* sprob, float* negent,
-                           uint8_t* rowmask, int Kp, uint32_t* header, cudaStream_t stream);
+// cache_format 0: int32 indices + fp32 logits; 1: uint16 indices + bf16 logits.
+cudaError_t launch_prepass(int cache_format, const void* topk_idx, const void* topk_logit, const uint8_t* mask,
+                           const int32_t* labels, int64_t N, int32_t V, int32_t K, float tau, float gamma,
+                           float beta, int* sidx, float* sprob, float* negent, float* wsum, uint8_t* rowmask,
+                           int Kp, uint32_t* header, cudaStream_t stream);
 
 cudaError_t launch_merge(const float* part_m, const float* part_s, const float* part_a, int splits,
-                         int rows_per_block, const float* negent, const uint8_t* rowmask, int64_t N, float* lse,
-                         float* loss, double* blocksum, uint32_t* header, cudaStream_t stream);
+                         int rows_per_block, float student_tau, const float* negent, const float* wsum,
+                         const uint8_t* rowmask, int64_t N, float* lse, float* loss, double* blocksum,
+                         uint32_t* header, cudaStream_t stream);
 
 // GEMM kinds: A/B majorness and epilogue are fixed per kind.
 //   kEpiLse      : A = hidden K-major, B = W K-major, BN = 256, row-stream

@@ -30,18 +30,35 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 // ============================================================================
 // prepass: one warp per row
+//
+// Builds each row's target list: the teacher's cached entries with indices
+// outside [0, V) dropped, sorted by index, repeats merged, probabilities
+// gamma * softmax(logit / tau), plus beta at the row's hard label when one is
+// given (merged into the cached entry of the same index, or inserted).  Also
+// writes gamma * sum P_T log P_T, the list's total weight, the effective mask,
+// N_valid and the data-error flags.
 // ============================================================================
 constexpr int kPreWarps = 8;
+constexpr int kListMax = kMaxK + 4;   // cached entries + the label, with room to spare
 
+__device__ __forceinline__ int load_idx(const int32_t* p, int64_t i) { return p[i]; }
+__device__ __forceinline__ int load_idx(const uint16_t* p, int64_t i) { return static_cast<int>(p[i]); }
+__device__ __forceinline__ float load_logit(const float* p, int64_t i) { return p[i]; }
+__device__ __forceinline__ float load_logit(const uint16_t* p, int64_t i) {
+  return __uint_as_float(static_cast<uint32_t>(p[i]) << 16);   // bf16 -> fp32, exact
+}
+
+template <typename IdxT, typename LogitT>
 __global__ void __launch_bounds__(kPreWarps * 32)
-    prepass_kernel(const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_logit,
-                   const uint8_t* __restrict__ mask, int64_t N, int V, int K, float inv_tau,
-                   int* __restrict__ sidx, float* __restrict__ sprob, float* __restrict__ negent,
-                   uint8_t* __restrict__ rowmask, int Kp, uint32_t* __restrict__ header) {
-  __shared__ int s_key[kPreWarps][kMaxK];
-  __shared__ float s_p[kPreWarps][kMaxK];
-  __shared__ int s_skey[kPreWarps][kMaxK];
-  __shared__ float s_sp[kPreWarps][kMaxK];
+    prepass_kernel(const IdxT* __restrict__ topk_idx, const LogitT* __restrict__ topk_logit,
+                   const uint8_t* __restrict__ mask, const int32_t* __restrict__ labels, int64_t N, int V, int K,
+                   float inv_tau, float gamma, float beta, int* __restrict__ sidx, float* __restrict__ sprob,
+                   float* __restrict__ negent, float* __restrict__ wsum, uint8_t* __restrict__ rowmask, int Kp,
+                   uint32_t* __restrict__ header) {
+  __shared__ int s_key[kPreWarps][kListMax];
+  __shared__ float s_p[kPreWarps][kListMax];
+  __shared__ int s_skey[kPreWarps][kListMax];
+  __shared__ float s_sp[kPreWarps][kListMax];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int* key = s_key[w];
   float* pv = s_p[w];
@@ -51,8 +68,7 @@ __global__ void __launch_bounds__(kPreWarps * 32)
   uint32_t wvalid = 0;
   const int64_t warps_total = static_cast<int64_t>(gridDim.x) * kPreWarps;
   for (int64_t n = static_cast<int64_t>(blockIdx.x) * kPreWarps + w; n < N; n += warps_total) {
-    const int32_t* ip = topk_idx + n * K;
-    const float* lp = topk_logit + n * K;
+    const int64_t base_in = n * K;
     int ki[8];
     float xi[8];
     bool keep[8];
@@ -65,8 +81,8 @@ __global__ void __launch_bounds__(kPreWarps * 32)
       xi[i] = -INFINITY;
       keep[i] = false;
       if (k < K) {
-        const int id = ip[k];
-        const float x = lp[k] * inv_tau;
+        const int id = load_idx(topk_idx, base_in + k);
+        const float x = load_logit(topk_logit, base_in + k) * inv_tau;
         keep[i] = (id >= 0) && (id < V);
         ki[i] = id;
         xi[i] = x;
@@ -95,6 +111,7 @@ __global__ void __launch_bounds__(kPreWarps * 32)
       }
       if (lane == 0) {
         negent[n] = 0.f;
+        wsum[n] = 0.f;
         rowmask[n] = 0;
       }
       __syncwarp();
@@ -136,9 +153,9 @@ __global__ void __launch_bounds__(kPreWarps * 32)
       }
     }
     __syncwarp();
-    // merge runs of equal indices, compact, and sum P log P
+    // merge runs of equal indices, compact into key/pv, and sum P log P
     float ent = 0.f;
-    int base = 0;
+    int cnt = 0;
     bool dup = false;
     for (int r0 = 0; r0 < K; r0 += 32) {
       const int r = r0 + lane;
@@ -157,23 +174,55 @@ __global__ void __launch_bounds__(kPreWarps * 32)
         }
       }
       const uint32_t ballot = __ballot_sync(0xffffffffu, start);
-      const int pos = base + __popc(ballot & ((1u << lane) - 1u));
+      const int pos = cnt + __popc(ballot & ((1u << lane) - 1u));
       if (start) {
-        out_i[pos] = kk;
-        out_p[pos] = pm;
+        key[pos] = kk;
+        pv[pos] = gamma * pm;
         if (pm > 0.f) ent += pm * logf(pm);
       }
-      base += __popc(ballot);
+      cnt += __popc(ballot);
     }
-    for (int k = base + lane; k < Kp; k += 32) {
-      out_i[k] = kSentinel;
-      out_p[k] = 0.f;
+    __syncwarp();
+    // the hard label joins the list with weight beta
+    float wrow = gamma;
+    if (labels != nullptr && beta != 0.f) {
+      const int lab = labels[n];
+      if (lab >= 0 && lab < V) {
+        wrow += beta;
+        int grew = 0;
+        if (lane == 0) {
+          int lo = 0, hi = cnt;
+          while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (key[mid] < lab) lo = mid + 1;
+            else hi = mid;
+          }
+          if (lo < cnt && key[lo] == lab) {
+            pv[lo] += beta;
+          } else {
+            for (int t = cnt; t > lo; --t) {
+              key[t] = key[t - 1];
+              pv[t] = pv[t - 1];
+            }
+            key[lo] = lab;
+            pv[lo] = beta;
+            grew = 1;
+          }
+        }
+        cnt += __shfl_sync(0xffffffffu, grew, 0);
+        __syncwarp();
+      }
+    }
+    for (int k = lane; k < Kp; k += 32) {
+      out_i[k] = k < cnt ? key[k] : kSentinel;
+      out_p[k] = k < cnt ? pv[k] : 0.f;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ent += __shfl_xor_sync(0xffffffffu, ent, o);
     if (__any_sync(0xffffffffu, dup)) wflags |= 2u;
     if (lane == 0) {
-      negent[n] = ent;
+      negent[n] = gamma * ent;
+      wsum[n] = wrow;
       const uint8_t m = (mask[n] != 0) ? 1 : 0;
       rowmask[n] = m;
       wvalid += m;
@@ -186,16 +235,23 @@ __global__ void __launch_bounds__(kPreWarps * 32)
   }
 }
 
-cudaError_t launch_prepass(const int32_t* topk_idx, const float* topk_logit, const uint8_t* mask, int64_t N,
-                           int32_t V, int32_t K, float tau, int* sidx, float* sprob, float* negent,
-                           uint8_t* rowmask, int Kp, uint32_t* header, cudaStream_t stream) {
+cudaError_t launch_prepass(int cache_format, const void* topk_idx, const void* topk_logit, const uint8_t* mask,
+                           const int32_t* labels, int64_t N, int32_t V, int32_t K, float tau, float gamma,
+                           float beta, int* sidx, float* sprob, float* negent, float* wsum, uint8_t* rowmask,
+                           int Kp, uint32_t* header, cudaStream_t stream) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t want = (N + kPreWarps - 1) / kPreWarps;
   const int grid = static_cast<int>(want < static_cast<int64_t>(sms) * 8 ? want : static_cast<int64_t>(sms) * 8);
-  prepass_kernel<<<grid, kPreWarps * 32, 0, stream>>>(topk_idx, topk_logit, mask, N, V, K, 1.0f / tau, sidx,
-                                                       sprob, negent, rowmask, Kp, header);
+  if (cache_format == 1)
+    prepass_kernel<uint16_t, uint16_t><<<grid, kPreWarps * 32, 0, stream>>>(
+        static_cast<const uint16_t*>(topk_idx), static_cast<const uint16_t*>(topk_logit), mask, labels, N, V, K,
+        1.0f / tau, gamma, beta, sidx, sprob, negent, wsum, rowmask, Kp, header);
+  else
+    prepass_kernel<int32_t, float><<<grid, kPreWarps * 32, 0, stream>>>(
+        static_cast<const int32_t*>(topk_idx), static_cast<const float*>(topk_logit), mask, labels, N, V, K,
+        1.0f / tau, gamma, beta, sidx, sprob, negent, wsum, rowmask, Kp, header);
   return cudaGetLastError();
 }
 
@@ -206,9 +262,9 @@ constexpr int kMergeThreads = 256;
 
 __global__ void __launch_bounds__(kMergeThreads)
     merge_kernel(const float* __restrict__ part_m, const float* __restrict__ part_s,
-                 const float* __restrict__ part_a, int splits, int rows_per_block,
-                 const float* __restrict__ negent, const uint8_t* __restrict__ rowmask, int64_t N,
-                 float* __restrict__ lse,
+                 const float* __restrict__ part_a, int splits, int rows_per_block, float inv_tau_s,
+                 const float* __restrict__ negent, const float* __restrict__ wsum,
+                 const uint8_t* __restrict__ rowmask, int64_t N, float* __restrict__ lse,
                  float* __restrict__ loss, double* __restrict__ blocksum, uint32_t* __restrict__ header) {
   __shared__ double s_red[kMergeThreads / 32];
   __shared__ bool s_last;
@@ -222,12 +278,15 @@ __global__ void __launch_bounds__(kMergeThreads)
     float s = 0.f, a = 0.f;
     for (int j = 0; j < splits; ++j) {
       const int64_t slot = (rb * splits + j) * rows_per_block + r;
-      s += part_s[slot] * expf(part_m[slot] - M);
+      s += part_s[slot] * expf((part_m[slot] - M) * inv_tau_s);
       a += part_a[slot];
     }
-    const float l = M + logf(s);
+    // lse of z / tau_s; the row's loss is gamma sum P_T log P_T - sum target * z / tau_s + weight * lse
+    const float l = M * inv_tau_s + logf(s);
     lse[n] = l;
-    if (rowmask[n]) kl = static_cast<double>(negent[n]) - static_cast<double>(a) + static_cast<double>(l);
+    if (rowmask[n])
+      kl = static_cast<double>(negent[n]) - static_cast<double>(a) * inv_tau_s +
+           static_cast<double>(wsum[n]) * static_cast<double>(l);
   }
   // block tree reduction (fixed order)
 #pragma unroll
@@ -255,11 +314,13 @@ __global__ void __launch_bounds__(kMergeThreads)
 }
 
 cudaError_t launch_merge(const float* part_m, const float* part_s, const float* part_a, int splits,
-                         int rows_per_block, const float* negent, const uint8_t* rowmask, int64_t N, float* lse,
-                         float* loss, double* blocksum, uint32_t* header, cudaStream_t stream) {
+                         int rows_per_block, float student_tau, const float* negent, const float* wsum,
+                         const uint8_t* rowmask, int64_t N, float* lse, float* loss, double* blocksum,
+                         uint32_t* header, cudaStream_t stream) {
   const int grid = static_cast<int>((N + kMergeThreads - 1) / kMergeThreads);
-  merge_kernel<<<grid, kMergeThreads, 0, stream>>>(part_m, part_s, part_a, splits, rows_per_block, negent, rowmask,
-                                                   N, lse, loss, blocksum, header);
+  merge_kernel<<<grid, kMergeThreads, 0, stream>>>(part_m, part_s, part_a, splits, rows_per_block,
+                                                   1.0f / student_tau, negent, wsum, rowmask, N, lse, loss,
+                                                   blocksum, header);
   return cudaGetLastError();
 }
 
@@ -521,10 +582,12 @@ __global__ void __launch_bounds__(192, 1)
     uint32_t acc_phase = 0;
     float g_scale = 0.f;
     if (KIND == kEpiGrad) {
+      // d loss / d z = (g / (tau_s N_valid)) (weight P_S - target)
       const uint32_t nv = *ep.n_valid;
       const float g = ep.grad_loss ? *ep.grad_loss : 1.0f;
-      g_scale = nv > 0 ? g / static_cast<float>(nv) : 0.f;
+      g_scale = nv > 0 ? g * ep.inv_tau_s / static_cast<float>(nv) : 0.f;
     }
+    const float es = ep.exp_scale;   // log2(e) / tau_s
     uint8_t* wbuf = sEpi + (warp - 2) * 4096;   // this warp's staging (grad: 2 x 2 KB, dW: 4 KB)
     int sbuf = 0;
     for (int u = group; u < sc.units; u += ngroups) {
@@ -536,7 +599,7 @@ __global__ void __launch_bounds__(192, 1)
       const int64_t grow = ep.row_offset + row;
       // per-row state of the loss epilogues
       float m_run = -INFINITY, s_run = 0.f, a_run = 0.f;
-      float cn = 0.f, lse_l2 = INFINITY;
+      float cn = 0.f, cnw = 0.f, lse_l2 = INFINITY;
       int kpos = 0, nxt = kSentinel;
       float nxtp = 0.f;
       const int* lst = nullptr;
@@ -546,7 +609,10 @@ __global__ void __launch_bounds__(192, 1)
         if (KIND == kEpiGrad) {
           cn = (rv && ep.rowmask[grow]) ? g_scale : 0.f;
           live = (cn != 0.f);
-          if (live) lse_l2 = ep.lse[grow] * kLog2e;
+          if (live) {
+            lse_l2 = ep.lse[grow] * kLog2e;
+            cnw = cn * ep.wsum[grow];
+          }
         }
         if (live) {
           lst = ep.sidx + grow * ep.Kp;
@@ -577,11 +643,11 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
             for (int j = 1; j < 32; ++j) cm = fmaxf(cm, v[j]);
             const float mn = fmaxf(m_run, cm);
-            const float ms = mn * kLog2e;
+            const float ms = mn * es;
             float acc_s = 0.f;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) acc_s += ex2_approx(fmaf(v[j], kLog2e, -ms));
-            s_run = s_run * ex2_approx((m_run - mn) * kLog2e) + acc_s;
+            for (int j = 0; j < 32; ++j) acc_s += ex2_approx(fmaf(v[j], es, -ms));
+            s_run = s_run * ex2_approx((m_run - mn) * es) + acc_s;
             m_run = mn;
             while (nxt < col + 32) {
               a_run = fmaf(nxtp, pick32(v, static_cast<uint32_t>(nxt - col)), a_run);
@@ -592,7 +658,7 @@ __global__ void __launch_bounds__(192, 1)
           } else if (KIND == kEpiGrad) {
             float g[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) g[j] = cn * ex2_approx(fmaf(v[j], kLog2e, -lse_l2));
+            for (int j = 0; j < 32; ++j) g[j] = cnw * ex2_approx(fmaf(v[j], es, -lse_l2));
             while (nxt < col + 32) {
               const uint32_t off = static_cast<uint32_t>(nxt - col);
               const float cp = cn * nxtp;

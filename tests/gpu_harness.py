@@ -37,22 +37,30 @@ class GpuResult:
     flags: int
 
 
-def run_gpu(dx: DevInputs, *, chunk_tokens=0, grad_loss=None, backward=True) -> GpuResult:
+def run_gpu(dx: DevInputs, *, chunk_tokens=0, grad_loss=None, backward=True, options=None) -> GpuResult:
+    """Forward (+ backward) through the C ABI; `options` (kdkl_options) selects the _ex entry points."""
     N, d = dx.hidden.shape
     V = dx.W.shape[0]
     Kc = dx.idx.shape[1]
     ws = torch.empty(K.kdkl_workspace_bytes(N, d, V, Kc, chunk_tokens), dtype=torch.uint8, device="cuda")
     loss = torch.full((1,), float("nan"), dtype=torch.float32, device="cuda")
     lse = torch.full((N,), float("nan"), dtype=torch.float32, device="cuda")
-    K.kdkl_forward(dx.hidden, dx.W, dx.idx, dx.logit, dx.mask, dx.tau, loss, lse, ws)
+    if options is None:
+        K.kdkl_forward(dx.hidden, dx.W, dx.idx, dx.logit, dx.mask, dx.tau, loss, lse, ws)
+    else:
+        K.kdkl_forward_ex(dx.hidden, dx.W, dx.idx, dx.logit, dx.mask, dx.tau, loss, lse, ws, options)
     flags = K.kdkl_read_device_flags(ws)
     dH = dW = None
     if backward:
         dHt = torch.full((N, d), float("nan"), dtype=torch.bfloat16, device="cuda")
         dWt = torch.full((V, d), float("nan"), dtype=torch.float32, device="cuda")
         g = None if grad_loss is None else torch.tensor([grad_loss], dtype=torch.float32, device="cuda")
-        K.kdkl_backward(dx.hidden, dx.W, dx.idx, dx.logit, dx.mask, dx.tau, lse, g, dHt, dWt, ws,
-                        chunk_tokens=chunk_tokens)
+        if options is None:
+            K.kdkl_backward(dx.hidden, dx.W, dx.idx, dx.logit, dx.mask, dx.tau, lse, g, dHt, dWt, ws,
+                            chunk_tokens=chunk_tokens)
+        else:
+            K.kdkl_backward_ex(dx.hidden, dx.W, dx.idx, dx.logit, dx.mask, dx.tau, lse, g, dHt, dWt, ws, options,
+                               chunk_tokens=chunk_tokens)
         flags |= K.kdkl_read_device_flags(ws)
         dH = dHt.float().cpu().numpy().astype(np.float64)
         dW = dWt.cpu().numpy().astype(np.float64)

@@ -1,0 +1,92 @@
+"""CUDA path vs the oracle for the compact cache format (uint16 indices + bf16
+logits) and the loss-design variants (student temperature, tau^2 factor,
+hard-label cross-entropy term), on seeded inputs with ragged tails."""
+import numpy as np
+import pytest
+import torch
+
+import output_head_kl_b200 as K
+import synth
+from oracle import kl as O
+from tests import gpu_harness as H
+
+pytestmark = pytest.mark.gpu
+
+
+def _compact(x):
+    """The same cache stored as uint16 indices and bf16 logits, and its exact widening."""
+    idx16 = x.topk_idx.astype(np.uint16)
+    lg16 = synth.f32_to_bf16_bits(x.topk_logit)
+    widened = synth.Inputs(x.hidden_bits, x.W_bits, idx16.astype(np.int32),
+                           O.bf16_bits_to_f64(lg16).astype(np.float32), x.mask, x.tau)
+    return idx16, lg16, widened
+
+
+def _parity(g, r):
+    assert g.flags == r.flags
+    H.assert_loss(g.loss, r.loss)
+    H.assert_lse(g.lse, r.lse)
+    H.assert_grad(g.dH, r.dH, "dHidden")
+    H.assert_grad(g.dW, r.dW, "dW")
+
+
+def test_compact_cache_matches_oracle_and_wide_cache():
+    x = synth.custom_inputs(700, 192, 3001, 24, seed=301, cache="zipf", logit_std=3.0, mask_frac=0.05, w_std=0.05)
+    idx16, lg16, wide = _compact(x)
+    dx = H.to_device(wide)
+    g_wide = H.run_gpu(dx, chunk_tokens=256)
+    dx16 = H.to_device(wide)
+    dx16.idx = torch.from_numpy(idx16.view(np.int16)).cuda()
+    dx16.logit = torch.from_numpy(lg16.view(np.int16)).cuda()
+    g16 = H.run_gpu(dx16, chunk_tokens=256, options=K.kdkl_options(cache_format=K.CACHE_U16_BF16))
+    r = O.kl_loss(wide.hidden_bits, wide.W_bits, wide.topk_idx, wide.topk_logit, wide.mask, wide.tau)
+    _parity(g16, r)
+    assert g16.loss == g_wide.loss
+    np.testing.assert_array_equal(g16.lse, g_wide.lse)
+    np.testing.assert_array_equal(g16.dH, g_wide.dH)
+    np.testing.assert_array_equal(g16.dW, g_wide.dW)
+
+
+def test_compact_cache_rejects_large_vocab():
+    x = synth.custom_inputs(4, 16, 70000, 2, seed=302)
+    dx = H.to_device(x)
+    ws = torch.empty(K.kdkl_workspace_bytes(4, 16, 70000, 2), dtype=torch.uint8, device="cuda")
+    loss = torch.empty(1, device="cuda")
+    lse = torch.empty(4, device="cuda")
+    st = K.kdkl_forward_ex(dx.hidden, dx.W, dx.idx, dx.logit, dx.mask, 1.0, loss, lse, ws,
+                           K.kdkl_options(cache_format=K.CACHE_U16_BF16), check=False)
+    assert st == 2 and "65536" in K.kdkl_last_error()
+
+
+VARIANTS = [
+    (O.Variant(student_tau=2.0, kd_scale_tau_sq=True), 2.0),
+    (O.Variant(student_tau=1.5, kd_weight=0.6, ce_weight=0.4), 1.0),
+    (O.Variant(kd_weight=0.0, ce_weight=1.0), 1.0),
+    (O.Variant(student_tau=0.7, kd_weight=0.3, kd_scale_tau_sq=True, ce_weight=2.0), 1.0),
+]
+
+
+@pytest.mark.parametrize("variant,tau", VARIANTS)
+def test_loss_variants_match_oracle(variant, tau):
+    x = synth.custom_inputs(600, 200, 2500, 20, seed=303, tau=tau, cache="zipf", logit_std=3.0, mask_frac=0.05,
+                            w_std=0.08)
+    rng = np.random.default_rng(304)
+    lab = rng.integers(0, 2500, size=600).astype(np.int32)
+    lab[rng.random(600) < 0.1] = -100
+    lab[:40] = x.topk_idx[:40, 0]            # labels that coincide with a cached entry
+    dx = H.to_device(x)
+    labels = torch.from_numpy(lab).cuda()
+    opts = K.kdkl_options(student_tau=variant.student_tau, kd_weight=variant.kd_weight,
+                          kd_scale_tau_sq=variant.kd_scale_tau_sq, ce_weight=variant.ce_weight, labels=labels)
+    g = H.run_gpu(dx, chunk_tokens=256, options=opts)
+    r = O.kl_loss(x.hidden_bits, x.W_bits, x.topk_idx, x.topk_logit, x.mask, x.tau, variant=variant, labels=lab)
+    _parity(g, r)
+
+
+def test_default_options_equal_plain_entry_points():
+    x = synth.custom_inputs(300, 128, 1500, 8, seed=305, mask_frac=0.1, w_std=0.1)
+    dx = H.to_device(x)
+    a = H.run_gpu(dx)
+    b = H.run_gpu(dx, options=K.kdkl_options())
+    assert a.loss == b.loss
+    np.testing.assert_array_equal(a.dW, b.dW)
