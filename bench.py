@@ -42,6 +42,67 @@ def measured_peaks():
     return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
 
 
+# ----------------------------------------------------------------------------- ncu traffic record
+def kernel_sources_digest() -> str:
+    """sha256 over the CUDA sources; a traffic record only applies to the kernels it was taken on."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "output_head_kl_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(workload: str, kernel: str):
+    """DRAM bytes (read + write) per launch from the committed ncu record, or None if stale/absent."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    if rec.get("sources_sha256") != kernel_sources_digest():
+        return None
+    entry = rec.get("workloads", {}).get(workload, {}).get(kernel)
+    return None if entry is None else float(entry["dram_bytes_per_launch"])
+
+
+_NCU_KIND = {"0": "fwd_lse_gemm", "1": "bwd_grad_gemm", "2": "bwd_dhidden_gemm", "3": "bwd_dw_gemm",
+             "4": "teacher_topk_gemm"}
+
+
+def record_traffic(csv_path: str, workload: str) -> dict:
+    """Writes profiles/traffic.json from an ncu --csv log of dram__bytes_{read,write}.sum (per-launch mean)."""
+    import csv
+    import re
+    rows = list(csv.reader(open(csv_path)))
+    head = next(i for i, r in enumerate(rows) if r and r[0] == "ID")
+    hdr = rows[head]
+    kname, mname, mval = hdr.index("Kernel Name"), hdr.index("Metric Name"), hdr.index("Metric Value")
+    per_launch = {}
+    for r in rows[head + 1:]:
+        if len(r) <= mval or not r[mname].startswith("dram__bytes_"):
+            continue
+        m = re.search(r"gemm_kernel<(\d+)", r[kname])
+        if not m:
+            continue
+        key = (_NCU_KIND[m.group(1)], r[0])
+        per_launch[key] = per_launch.get(key, 0.0) + float(r[mval].replace(",", ""))
+    sums = {}
+    for (kind, _), b in per_launch.items():
+        sums.setdefault(kind, []).append(b)
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    rec = json.load(open(p)) if os.path.exists(p) else {}
+    if rec.get("sources_sha256") != kernel_sources_digest():
+        rec = {"sources_sha256": kernel_sources_digest(), "workloads": {}}
+    rec["workloads"][workload] = {k: {"dram_bytes_per_launch": sum(v) / len(v), "launches_captured": len(v)}
+                                  for k, v in sums.items()}
+    with open(p, "w") as f:
+        json.dump(rec, f, indent=1, sort_keys=True)
+    return rec
+
+
 # ----------------------------------------------------------------------------- clocks
 _REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
                 0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
@@ -277,7 +338,7 @@ def main_gpu(args, w: synth.Workload, N: int):
     # (hidden, cache, mask) goes host -> device from pinned memory and the
     # loss comes back device -> host
     h_loss = torch.empty(1, dtype=torch.float32).pin_memory()
-    e2e_steps = max(1, min(args.steps, 5))
+    e2e_steps = args.steps
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -315,7 +376,7 @@ def main_gpu(args, w: synth.Workload, N: int):
                     "peak_kind": f"bf16 dense, sustained ({peaks['source']})",
                     "frac_of_burst_peak": achieved / peaks["bf16_tflops"],
                     "flops_per_launch": alg, "avg_launch_ms": total_ms / launches,
-                    "traffic": None}
+                    "traffic": recorded_traffic(w.name, dom)}
         else:
             roof = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": None, "traffic": None}
@@ -357,6 +418,59 @@ def main_gpu(args, w: synth.Workload, N: int):
     return 0
 
 
+def main_topk(args, w: synth.Workload, N: int):
+    """Teacher top-K cache producer: z = hidden W^T (2 N d V flops) + per-row top-K (K = the workload's K)."""
+    import torch
+
+    import output_head_kl_b200 as K
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    K.lib()
+    x = synth.make_inputs(w, N=N)
+    Nn, d, V, Kc = x.shape
+
+    def bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    hidden, W = bf16(x.hidden_bits), bf16(x.W_bits)
+    ws = torch.empty(K.kdkl_teacher_topk_workspace_bytes(Nn, d, V, Kc), dtype=torch.uint8, device=dev)
+    idx = torch.empty(Nn, Kc, dtype=torch.int32, device=dev)
+    val = torch.empty(Nn, Kc, dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        K.kdkl_teacher_topk(hidden, W, Kc, idx, val, ws)
+    torch.cuda.synchronize()
+    K.kdkl_timing_read(reset=True)
+    sampler = ClockSampler(gpu_id_for(0))
+    sampler.start()
+    time.sleep(0.3)
+    K.kdkl_timing_enable(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        K.kdkl_teacher_topk(hidden, W, Kc, idx, val, ws)
+    e1.record()
+    torch.cuda.synchronize()
+    K.kdkl_timing_enable(False)
+    kt = K.kdkl_timing_read(reset=True)
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    peaks = measured_peaks()
+    launches, total = kt["teacher_topk_gemm"]
+    achieved = 2.0 * Nn * d * V / (total / launches * 1e-3) / 1e12
+    print(json.dumps({
+        "metric": "teacher top-K cache producer tokens/sec", "value": Nn / (ms * 1e-3), "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name + "_teacher_topk", "N": Nn, "d": d, "V": V, "K": Kc},
+        "tflops": 2.0 * Nn * d * V / (ms * 1e-3) / 1e12,
+        "roofline": {"kernel": "teacher_topk_gemm", "bound": "tensor", "achieved": achieved,
+                     "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops_sustained"], "traffic": None},
+        "kernels": {k: {"launches": v[0], "ms_per_step": v[1] / args.steps} for k, v in kt.items() if v[0]},
+        "gpu_launches": int(sum(v[0] for v in kt.values())), "clocks": clocks}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -367,13 +481,21 @@ def main():
     ap.add_argument("--N", type=int, default=None, help="token count override (sweep points)")
     ap.add_argument("--chunk-tokens", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--topk", action="store_true", help="time the teacher top-K cache producer instead")
+    ap.add_argument("--record-traffic", metavar="NCU_CSV",
+                    help="write profiles/traffic.json from an ncu dram__bytes capture of --config's workload")
     ap.add_argument("--sweep", action="store_true",
                     help="long-context sweep (d=4096, V=128256, tau=2): one JSON line per N, single GPU")
     args = ap.parse_args()
     w = synth.CONFIGS[args.config]
     N = args.N if args.N is not None else w.N
+    if args.record_traffic:
+        print(json.dumps(record_traffic(args.record_traffic, w.name)))
+        return 0
     if args.impl == "reference":
         return run_reference(args, w, N)
+    if args.topk:
+        return main_topk(args, w, N)
     if args.sweep:
         args.no_cpu_baseline = True
         for n in synth.SWEEP_N:

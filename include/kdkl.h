@@ -194,6 +194,26 @@ kdkl_status kdkl_backward_ex(const void* hidden, const void* W, const void* topk
                              size_t workspace_bytes, void* stream);
 
 /*
+ * Teacher top-K cache producer: the step that builds the cache the loss reads.
+ * The teacher runs once and, for each token position, only its K most likely
+ * vocabulary entries are kept as (index, logit) pairs (mind-verse.de article,
+ * section "Zwei systemische Optimierungen", item 1; llm-wiki note, section
+ * "사전 계산 파이프라인", steps 2-3).  Given the teacher's last hidden states and
+ * output head, this computes z = hidden W^T tile by tile on the tensor cores
+ * (never storing z) and keeps each row's K largest logits:
+ *   hidden      [N, d] bf16, 16-byte aligned; W [V, d] bf16, 16-byte aligned
+ *   1 <= K <= 128, K <= V, d % 8 == 0
+ *   topk_idx    [N, K] int32 out; topk_logit [N, K] fp32 out (the fp32 logits z)
+ *   each row ordered by logit descending, ties to the smaller index
+ *   workspace   >= kdkl_teacher_topk_workspace_bytes(N, d, V, K), 256-byte aligned
+ * The output is directly a KDKL_CACHE_I32_F32 cache for kdkl_forward.
+ */
+size_t kdkl_teacher_topk_workspace_bytes(int64_t N, int32_t d, int32_t V, int32_t K);
+kdkl_status kdkl_teacher_topk(const void* hidden, const void* W, int64_t N, int32_t d, int32_t V, int32_t K,
+                              int32_t* topk_idx, float* topk_logit, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/*
  * Reads the device flag word of the most recent forward/backward call that
  * used `workspace` (each call clears it first).  Synchronises `stream`.
  */
@@ -209,7 +229,8 @@ kdkl_status kdkl_read_device_flags(const void* workspace, void* stream, uint32_t
  * the totals afterwards.  Enabling costs two event records per launch.
  */
 typedef struct {
-  const char* name;   /* "prepass", "fwd_lse_gemm", "merge", "bwd_grad_gemm", "bwd_dhidden_gemm", "bwd_dw_gemm" */
+  const char* name;   /* "prepass", "fwd_lse_gemm", "merge", "bwd_grad_gemm", "bwd_dhidden_gemm", "bwd_dw_gemm",
+                         "teacher_topk_gemm", "teacher_topk_merge" */
   uint64_t launches;  /* launches timed since the last reset */
   double total_ms;    /* summed device time of those launches */
 } kdkl_kernel_time;

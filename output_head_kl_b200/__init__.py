@@ -7,7 +7,7 @@ raises.
 
 Names mirror the C entry points: ``kdkl_workspace_bytes``, ``kdkl_forward``,
 ``kdkl_backward``, ``kdkl_forward_ex``, ``kdkl_backward_ex`` (with ``kdkl_options``),
-``kdkl_forward_noalloc``, ``kdkl_read_device_flags``, ``kdkl_timing_enable``,
+``kdkl_forward_noalloc``, ``kdkl_teacher_topk``, ``kdkl_read_device_flags``, ``kdkl_timing_enable``,
 ``kdkl_timing_read``, ``kdkl_status_string``, ``kdkl_last_error``.  ``fused_kl_forward_backward`` is a convenience wrapper
 that allocates the outputs and the workspace with torch (the library itself
 never allocates).
@@ -90,6 +90,10 @@ def lib() -> ctypes.CDLL:
     L.kdkl_backward_ex.argtypes = [vp, vp, vp, vp, vp, i64, i32, i32, i32, f32, ctypes.POINTER(Options), vp, vp, vp,
                                    vp, i64, vp, sz, vp]
     L.kdkl_backward_ex.restype = ctypes.c_int
+    L.kdkl_teacher_topk_workspace_bytes.argtypes = [i64, i32, i32, i32]
+    L.kdkl_teacher_topk_workspace_bytes.restype = sz
+    L.kdkl_teacher_topk.argtypes = [vp, vp, i64, i32, i32, i32, vp, vp, vp, sz, vp]
+    L.kdkl_teacher_topk.restype = ctypes.c_int
     L.kdkl_timing_enable.argtypes = [ctypes.c_int]
     L.kdkl_timing_enable.restype = ctypes.c_int
     L.kdkl_timing_read.argtypes = [ctypes.POINTER(KernelTime), ctypes.c_int, ctypes.c_int]
@@ -197,6 +201,24 @@ def kdkl_backward_ex(hidden, W, topk_idx, topk_logit, mask, tau, lse, grad_loss,
                                 _ptr(dW), int(chunk_tokens), _ptr(workspace), int(wsb), _stream(stream))
     if check:
         _check(st, "kdkl_backward_ex")
+    return st
+
+
+def kdkl_teacher_topk_workspace_bytes(N: int, d: int, V: int, K: int) -> int:
+    return int(lib().kdkl_teacher_topk_workspace_bytes(N, d, V, K))
+
+
+def kdkl_teacher_topk(hidden, W, K, topk_idx, topk_logit, workspace, *, N=None, d=None, V=None,
+                      workspace_bytes=None, stream=None, check=True) -> int:
+    """Calls kdkl_teacher_topk: the K largest logits of hidden W^T per row, with indices."""
+    N = hidden.shape[0] if N is None else N
+    d = hidden.shape[1] if d is None else d
+    V = W.shape[0] if V is None else V
+    wsb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    st = lib().kdkl_teacher_topk(_ptr(hidden), _ptr(W), int(N), int(d), int(V), int(K), _ptr(topk_idx),
+                                 _ptr(topk_logit), _ptr(workspace), int(wsb), _stream(stream))
+    if check:
+        _check(st, "kdkl_teacher_topk")
     return st
 
 

@@ -248,9 +248,10 @@ kdkl_status cuda_fail(cudaError_t e, const char* what) {
 }
 
 // ---------------------------------------------------------------- timing
-enum TimedKind { kTPrepass = 0, kTFwd, kTMerge, kTGrad, kTDh, kTDw, kTKinds };
-const char* const kTimedNames[kTKinds] = {"prepass", "fwd_lse_gemm", "merge", "bwd_grad_gemm", "bwd_dhidden_gemm",
-                                          "bwd_dw_gemm"};
+enum TimedKind { kTPrepass = 0, kTFwd, kTMerge, kTGrad, kTDh, kTDw, kTTopK, kTTopKMerge, kTKinds };
+const char* const kTimedNames[kTKinds] = {"prepass",          "fwd_lse_gemm", "merge",         "bwd_grad_gemm",
+                                          "bwd_dhidden_gemm", "bwd_dw_gemm",  "teacher_topk_gemm",
+                                          "teacher_topk_merge"};
 struct TimingRec {
   int kind;
   cudaEvent_t a, b;
@@ -572,6 +573,92 @@ kdkl_status kdkl_backward_ex(const void* hidden, const void* W, const void* topk
 
 void kdkl_options_init(kdkl_options* options) {
   if (options) *options = default_options();
+}
+
+// ---------------------------------------------------------------- teacher top-K producer
+namespace {
+struct TopkLayout {
+  size_t header = 0, tv = 0, ti = 0, total = 0;
+  int s_cap = 1;
+};
+
+TopkLayout topk_layout(int64_t N, int32_t K) {
+  TopkLayout L;
+  L.s_cap = 1024 / K > 0 ? 1024 / K : 1;
+  // enough partial slots for either tile height (256-row pairs or 128-row CTAs)
+  const size_t slots = static_cast<size_t>((N + 255) / 256 + 1) * 256 * L.s_cap * K;
+  size_t off = 256;
+  L.tv = off;
+  off = align_up(off + slots * 4, 256);
+  L.ti = off;
+  off = align_up(off + slots * 4, 256);
+  L.total = off;
+  return L;
+}
+
+kdkl_status check_topk_shapes(int64_t N, int32_t d, int32_t V, int32_t K) {
+  if (N < 0 || N > kMaxRows) return fail(KDKL_ERR_SHAPE, "N=%lld outside [0, %lld]", (long long)N, (long long)kMaxRows);
+  if (d < 8 || d % 8 != 0) return fail(KDKL_ERR_SHAPE, "d=%d must be a positive multiple of 8", d);
+  if (V < 1 || V > kMaxV) return fail(KDKL_ERR_SHAPE, "V=%d outside [1, 2^30]", V);
+  if (K < 1 || K > kTopKMax || K > V) return fail(KDKL_ERR_SHAPE, "K=%d outside [1, min(%d, V)]", K, kTopKMax);
+  return KDKL_OK;
+}
+}  // namespace
+
+size_t kdkl_teacher_topk_workspace_bytes(int64_t N, int32_t d, int32_t V, int32_t K) {
+  if (check_topk_shapes(N, d, V, K) != KDKL_OK) return 0;
+  return topk_layout(N, K).total;
+}
+
+kdkl_status kdkl_teacher_topk(const void* hidden, const void* W, int64_t N, int32_t d, int32_t V, int32_t K,
+                              int32_t* topk_idx, float* topk_logit, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  kdkl_status st = check_topk_shapes(N, d, V, K);
+  if (st != KDKL_OK) return st;
+  if (!hidden || !W || !topk_idx || !topk_logit || !workspace)
+    return fail(KDKL_ERR_NULL, "hidden, W, topk_idx, topk_logit and workspace must be non-NULL");
+  if (!aligned(hidden, 16) || !aligned(W, 16)) return fail(KDKL_ERR_ALIGN, "hidden and W must be 16-byte aligned");
+  if (!aligned(topk_idx, 4) || !aligned(topk_logit, 4))
+    return fail(KDKL_ERR_ALIGN, "topk_idx and topk_logit must be 4-byte aligned");
+  if (!aligned(workspace, 256)) return fail(KDKL_ERR_ALIGN, "workspace must be 256-byte aligned");
+  const TopkLayout L = topk_layout(N, K);
+  if (workspace_bytes < L.total)
+    return fail(KDKL_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, L.total);
+  Device dv;
+  if ((st = current_device(dv)) != KDKL_OK) return st;
+  const Pairing pr = pairing(dv, 256);
+  if (!pr.pair) return fail(KDKL_ERR_UNSUPPORTED, "the top-K producer needs CTA pairs");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(workspace, 0, 256, s)) != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  if (N == 0) return ok();
+  const int64_t rb = (N + pr.rows - 1) / pr.rows;
+  const int vt = (V + 255) / 256;
+  const int splits = pick_splits(rb, vt, pr.groups, d, rb * L.s_cap, pr.rows);
+  Sched sc{static_cast<int>(rb * splits), splits, vt, (d + kBK - 1) / kBK, 1};
+  CUtensorMap tmA, tmB;
+  if (!make_map(&tmA, hidden, d, N, d, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tmB, W, d, V, d, kBK, pr.b_rows, CU_TENSOR_MAP_SWIZZLE_128B))
+    return fail(KDKL_ERR_CUDA, "cuTensorMapEncodeTiled failed (hidden/W)");
+  EpiParams ep;
+  std::memset(&ep, 0, sizeof(ep));
+  ep.M = static_cast<int>(N);
+  ep.Ncols = V;
+  ep.topk_K = K;
+  ep.part_tv = at<float>(workspace, L.tv);
+  ep.part_ti = at<int>(workspace, L.ti);
+  ep.flags = at<uint32_t>(workspace, 0);
+  ep.exp_scale = 1.4426950408889634f;
+  ep.inv_tau_s = 1.0f;
+  const int grid = pr.grid(sc.units);
+  if ((e = timed(kTTopK, s, [&] { return launch_gemm(kEpiTopK, 256, true, tmA, tmB, tmA, sc, ep, grid, s); })) !=
+      cudaSuccess)
+    return cuda_fail(e, "top-K GEMM launch");
+  if ((e = timed(kTTopKMerge, s, [&] {
+         return launch_topk_merge(ep.part_tv, ep.part_ti, splits, pr.rows, K, N, topk_idx, topk_logit, s);
+       })) != cudaSuccess)
+    return cuda_fail(e, "top-K merge launch");
+  return ok();
 }
 
 kdkl_status kdkl_timing_enable(int enable) {

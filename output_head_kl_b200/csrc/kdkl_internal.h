@@ -82,9 +82,17 @@ struct EpiParams {
   int ldo;             // row pitch (elements) of dH / dW
   int accumulate;      // dW: add into the existing values
   uint32_t* flags;     // device flag word
+  // teacher top-K producer: K per row, partial heaps [units * rows_per_unit, K]
+  int topk_K;
+  float* part_tv;
+  int* part_ti;
 };
 
-enum EpiKind { kEpiLse = 0, kEpiGrad = 1, kEpiStoreBf16 = 2, kEpiRmwF32 = 3 };
+enum EpiKind { kEpiLse = 0, kEpiGrad = 1, kEpiStoreBf16 = 2, kEpiRmwF32 = 3, kEpiTopK = 4 };
+
+// Teacher top-K producer: per-row min-heaps of up to kTopKMax entries live in
+// shared memory during the vocabulary sweep.
+constexpr int kTopKMax = 128;
 
 // Launchers (defined in kernels.cu).  Each returns cudaGetLastError() of its launch.
 // cache_format 0: int32 indices + fp32 logits; 1: uint16 indices + bf16 logits.
@@ -109,6 +117,11 @@ cudaError_t launch_merge(const float* part_m, const float* part_s, const float* 
 cudaError_t launch_gemm(int kind, int BN, bool pair, const CUtensorMap& tmA, const CUtensorMap& tmB,
                         const CUtensorMap& tmOut, const Sched& sched, const EpiParams& ep, int grid,
                         cudaStream_t stream);
+
+// Merges the per-split heaps of the top-K producer into each row's K entries,
+// ordered by (logit descending, index ascending).
+cudaError_t launch_topk_merge(const float* part_tv, const int* part_ti, int splits, int rows_per_block, int K,
+                              int64_t N, int32_t* topk_idx, float* topk_logit, cudaStream_t stream);
 
 // Sets the message kdkl_last_error() returns on this host thread.
 void set_last_error(const char* msg);

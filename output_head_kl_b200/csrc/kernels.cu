@@ -346,7 +346,8 @@ struct GemmCfg {
   static constexpr int kBBytes = kCtaN * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;               // landing in this CTA
   static constexpr int kTxBytes = (PAIR ? 2 : 1) * kStageBytes;       // counted on the MMA's barrier
-  static constexpr int kEpiBytes = (KIND == kEpiGrad || KIND == kEpiRmwF32) ? 4 * 4096 : 0;
+  static constexpr int kEpiBytes =
+      (KIND == kEpiGrad || KIND == kEpiRmwF32) ? 4 * 4096 : (KIND == kEpiTopK ? kTopKMax * kBM * 8 : 0);
   static constexpr int kBarBytes = 256;
   static constexpr int kSmemLimit = 232448;
   static constexpr int kStagesFit = (kSmemLimit - 1024 - kEpiBytes - kBarBytes) / kStageBytes;
@@ -589,6 +590,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     const float es = ep.exp_scale;   // log2(e) / tau_s
     uint8_t* wbuf = sEpi + (warp - 2) * 4096;   // this warp's staging (grad: 2 x 2 KB, dW: 4 KB)
+    uint8_t* wbuf_all = sEpi;                    // top-K heaps of all 128 rows
     int sbuf = 0;
     for (int u = group; u < sc.units; u += ngroups) {
       int mb, t0, t1;
@@ -596,6 +598,17 @@ __global__ void __launch_bounds__(192, 1)
       const int row0 = mb * C::kMmaM + static_cast<int>(rank) * kBM;   // first row of this CTA
       const int row = row0 + row_local;
       const bool rv = row < ep.M;
+      // teacher top-K: this thread's row owns column row_local of two [kTopKMax][128]
+      // shared arrays holding a min-heap ordered by (value, then larger index first)
+      float* hv = reinterpret_cast<float*>(wbuf_all) + row_local;
+      int* hi = reinterpret_cast<int*>(wbuf_all + kTopKMax * kBM * 4) + row_local;
+      float hroot = -INFINITY;
+      if (KIND == kEpiTopK) {
+        for (int k = 0; k < ep.topk_K; ++k) {
+          hv[k * kBM] = -INFINITY;
+          hi[k * kBM] = kSentinel;
+        }
+      }
       const int64_t grow = ep.row_offset + row;
       // per-row state of the loss epilogues
       float m_run = -INFINITY, s_run = 0.f, a_run = 0.f;
@@ -704,6 +717,48 @@ __global__ void __launch_bounds__(192, 1)
                 }
               }
             }
+          } else if (KIND == kEpiTopK) {
+            const int Kh = ep.topk_K;
+            // candidates above the current root (a stale root only admits extras,
+            // which the exact test below rejects), taken in column order
+            uint32_t cand = 0;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) cand |= (v[j] > hroot) ? (1u << j) : 0u;
+            if (col + 32 > ep.Ncols) cand &= (1u << (ep.Ncols - col)) - 1u;
+            while (cand) {
+              const int j = __ffs(cand) - 1;
+              cand &= cand - 1u;
+              const float val = pick32(v, static_cast<uint32_t>(j));
+              if (val > hroot) {
+                // replace the root (the smallest kept entry) and sift down; within a
+                // unit columns arrive in increasing order, so ties keep the earlier index
+                const int vi = col + j;
+                int pos = 0;
+                while (true) {
+                  const int l = 2 * pos + 1;
+                  if (l >= Kh) break;
+                  int c = l;
+                  float cv = hv[l * kBM];
+                  int ci = hi[l * kBM];
+                  if (l + 1 < Kh) {
+                    const float rv2 = hv[(l + 1) * kBM];
+                    const int ri2 = hi[(l + 1) * kBM];
+                    if (rv2 < cv || (rv2 == cv && ri2 > ci)) {
+                      c = l + 1;
+                      cv = rv2;
+                      ci = ri2;
+                    }
+                  }
+                  if (cv > val || (cv == val && ci < vi)) break;   // child ranks above the new entry
+                  hv[pos * kBM] = cv;
+                  hi[pos * kBM] = ci;
+                  pos = c;
+                }
+                hv[pos * kBM] = val;
+                hi[pos * kBM] = vi;
+                hroot = hv[0];
+              }
+            }
           } else {  // kEpiRmwF32
             // Transpose the warp's 32 x 32 fp32 block through shared memory so
             // that each global access is one full 128-byte row segment.
@@ -743,6 +798,14 @@ __global__ void __launch_bounds__(192, 1)
         }
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
+      }
+      if (KIND == kEpiTopK && rv) {
+        const int64_t slot = (static_cast<int64_t>(u) * C::kMmaM + static_cast<int>(rank) * kBM + row_local) *
+                             ep.topk_K;
+        for (int k = 0; k < ep.topk_K; ++k) {
+          ep.part_tv[slot + k] = hv[k * kBM];
+          ep.part_ti[slot + k] = hi[k * kBM];
+        }
       }
       if (KIND == kEpiLse && rv) {
         const int64_t slot = static_cast<int64_t>(u) * C::kMmaM + static_cast<int>(rank) * kBM + row_local;
@@ -814,6 +877,7 @@ cudaError_t launch_gemm(int kind, int BN, bool pair, const CUtensorMap& tmA, con
       case kEpiGrad: return launch_one<kEpiGrad, 256, true>(tmA, tmB, tmOut, sc, ep, grid, stream);
       case kEpiStoreBf16: return launch_one<kEpiStoreBf16, 256, true>(tmA, tmB, tmOut, sc, ep, grid, stream);
       case kEpiRmwF32: return launch_one<kEpiRmwF32, 256, true>(tmA, tmB, tmOut, sc, ep, grid, stream);
+      case kEpiTopK: return launch_one<kEpiTopK, 256, true>(tmA, tmB, tmOut, sc, ep, grid, stream);
       default: return cudaErrorInvalidValue;
     }
   }
@@ -836,6 +900,83 @@ cudaError_t launch_gemm(int kind, int BN, bool pair, const CUtensorMap& tmA, con
       break;
   }
   return cudaErrorInvalidValue;
+}
+
+// ============================================================================
+// top-K merge: one warp per row sorts the row's split heaps (bitonic, in
+// shared memory) by (value descending, index ascending) and keeps the first K
+// ============================================================================
+constexpr int kMergeCand = 1024;   // splits * K never exceeds this (the planner caps splits)
+constexpr int kTopKMergeWarps = 4;
+
+__device__ __forceinline__ bool ranks_before(float av, int ai, float bv, int bi) {
+  return av > bv || (av == bv && ai < bi);
+}
+
+__global__ void __launch_bounds__(kTopKMergeWarps * 32)
+    topk_merge_kernel(const float* __restrict__ part_tv, const int* __restrict__ part_ti, int splits,
+                      int rows_per_block, int K, int64_t N, int32_t* __restrict__ topk_idx,
+                      float* __restrict__ topk_logit) {
+  __shared__ float s_v[kTopKMergeWarps][kMergeCand];
+  __shared__ int s_i[kTopKMergeWarps][kMergeCand];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* sv = s_v[w];
+  int* si = s_i[w];
+  const int C = splits * K;
+  int P = 32;
+  while (P < C) P <<= 1;
+  for (int64_t n = static_cast<int64_t>(blockIdx.x) * kTopKMergeWarps + w; n < N;
+       n += static_cast<int64_t>(gridDim.x) * kTopKMergeWarps) {
+    const int64_t rb = n / rows_per_block;
+    const int r = static_cast<int>(n - rb * rows_per_block);
+    for (int c = lane; c < P; c += 32) {
+      if (c < C) {
+        const int j = c / K, k = c - j * K;
+        const int64_t slot = ((rb * splits + j) * rows_per_block + r) * K + k;
+        sv[c] = part_tv[slot];
+        si[c] = part_ti[slot];
+      } else {
+        sv[c] = -INFINITY;
+        si[c] = kSentinel;
+      }
+    }
+    __syncwarp();
+    for (int k2 = 2; k2 <= P; k2 <<= 1) {
+      for (int j2 = k2 >> 1; j2 > 0; j2 >>= 1) {
+        for (int i = lane; i < P; i += 32) {
+          const int l = i ^ j2;
+          if (l > i) {
+            const float a = sv[i], b = sv[l];
+            const int ai = si[i], bi = si[l];
+            const bool up = (i & k2) == 0;
+            const bool sw = up ? ranks_before(b, bi, a, ai) : ranks_before(a, ai, b, bi);
+            if (sw) {
+              sv[i] = b;
+              si[i] = bi;
+              sv[l] = a;
+              si[l] = ai;
+            }
+          }
+        }
+        __syncwarp();
+      }
+    }
+    for (int k = lane; k < K; k += 32) {
+      topk_logit[n * K + k] = sv[k];
+      topk_idx[n * K + k] = si[k];
+    }
+    __syncwarp();
+  }
+}
+
+cudaError_t launch_topk_merge(const float* part_tv, const int* part_ti, int splits, int rows_per_block, int K,
+                              int64_t N, int32_t* topk_idx, float* topk_logit, cudaStream_t stream) {
+  if (splits * K > kMergeCand) return cudaErrorInvalidValue;
+  const int64_t blocks = (N + kTopKMergeWarps - 1) / kTopKMergeWarps;
+  const int grid = static_cast<int>(blocks < 4096 ? blocks : 4096);
+  topk_merge_kernel<<<grid, kTopKMergeWarps * 32, 0, stream>>>(part_tv, part_ti, splits, rows_per_block, K, N,
+                                                                topk_idx, topk_logit);
+  return cudaGetLastError();
 }
 
 }  // namespace kdkl
