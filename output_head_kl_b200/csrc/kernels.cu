@@ -686,15 +686,12 @@ __global__ void __launch_bounds__(192, 1)
             if (lane == 0) bulk_wait_read<1>();
             __syncwarp();
             const uint32_t sw = static_cast<uint32_t>((lane >> 1) & 3);
+            const uint32_t row_addr = smem_u32(buf) + static_cast<uint32_t>(lane) * 64u;
 #pragma unroll
-            for (int c16 = 0; c16 < 4; ++c16) {
-              uint4 pk;
-              pk.x = pack_bf16x2(g[c16 * 8 + 0], g[c16 * 8 + 1]);
-              pk.y = pack_bf16x2(g[c16 * 8 + 2], g[c16 * 8 + 3]);
-              pk.z = pack_bf16x2(g[c16 * 8 + 4], g[c16 * 8 + 5]);
-              pk.w = pack_bf16x2(g[c16 * 8 + 6], g[c16 * 8 + 7]);
-              *reinterpret_cast<uint4*>(buf + lane * 64 + ((static_cast<uint32_t>(c16) ^ sw) << 4)) = pk;
-            }
+            for (int c16 = 0; c16 < 4; ++c16)
+              st_shared_v4(row_addr + ((static_cast<uint32_t>(c16) ^ sw) << 4),
+                           pack_bf16x2(g[c16 * 8 + 0], g[c16 * 8 + 1]), pack_bf16x2(g[c16 * 8 + 2], g[c16 * 8 + 3]),
+                           pack_bf16x2(g[c16 * 8 + 4], g[c16 * 8 + 5]), pack_bf16x2(g[c16 * 8 + 6], g[c16 * 8 + 7]));
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
@@ -763,18 +760,20 @@ __global__ void __launch_bounds__(192, 1)
             // Transpose the warp's 32 x 32 fp32 block through shared memory so
             // that each global access is one full 128-byte row segment.
             // 16-byte chunk q of row r sits at chunk (q ^ (r & 7)): conflict-free both ways.
-            float* fb = reinterpret_cast<float*>(wbuf);
+            const uint32_t fb = smem_u32(wbuf);
 #pragma unroll
             for (int q4 = 0; q4 < 8; ++q4)
-              *reinterpret_cast<float4*>(fb + lane * 32 + ((q4 ^ (lane & 7)) << 2)) =
-                  make_float4(v[q4 * 4 + 0], v[q4 * 4 + 1], v[q4 * 4 + 2], v[q4 * 4 + 3]);
+              st_shared_v4(fb + static_cast<uint32_t>(lane * 128 + ((q4 ^ (lane & 7)) << 4)),
+                           __float_as_uint(v[q4 * 4 + 0]), __float_as_uint(v[q4 * 4 + 1]),
+                           __float_as_uint(v[q4 * 4 + 2]), __float_as_uint(v[q4 * 4 + 3]));
             __syncwarp();
             const int wrow0 = row0 + q * 32;
             const bool cv = (col + lane) < ep.Ncols;
             float r[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i)
-              r[i] = fb[i * 32 + ((((lane >> 2) ^ (i & 7))) << 2) + (lane & 3)];
+              r[i] = ld_shared_f32(fb + static_cast<uint32_t>(i * 128 + (((lane >> 2) ^ (i & 7)) << 4) +
+                                                              (lane & 3) * 4));
             __syncwarp();
             float* base = ep.dW + static_cast<int64_t>(wrow0) * ep.ldo + col + lane;
             if (ep.accumulate) {

@@ -145,3 +145,16 @@ def test_constant_W_column_gives_zero_dH_column():
     g, r = _full_parity(x)
     assert np.abs(g.dH[:, 5]).max() <= 1e-2 * np.abs(g.dH).max()
     assert np.abs(r.dH[:, 5]).max() < 1e-15
+
+
+def test_largest_cache_K256():
+    """K = 256 (the largest cache the ABI takes; eight entries per prepass lane)."""
+    x = synth.custom_inputs(300, 128, 3000, 256, seed=111, cache="zipf", logit_std=3.0, mask_frac=0.05, w_std=0.1)
+    _full_parity(x)
+
+
+def test_ragged_cache_K255_with_duplicates():
+    x = synth.custom_inputs(200, 64, 2000, 255, seed=112, w_std=0.1)
+    x.topk_idx[5, 200] = x.topk_idx[5, 3]
+    g, r = _full_parity(x)
+    assert g.flags == O.FLAG_IDX_DUP

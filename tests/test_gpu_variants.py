@@ -90,3 +90,16 @@ def test_default_options_equal_plain_entry_points():
     b = H.run_gpu(dx, options=K.kdkl_options())
     assert a.loss == b.loss
     np.testing.assert_array_equal(a.dW, b.dW)
+
+
+def test_variant_with_full_cache_and_label_insertion():
+    """K = 256 cached entries plus a label per row: the target list holds 257 entries."""
+    x = synth.custom_inputs(260, 128, 3000, 256, seed=306, cache="zipf", logit_std=3.0, w_std=0.1)
+    rng = np.random.default_rng(307)
+    lab = rng.integers(0, 3000, size=260).astype(np.int32)
+    v = O.Variant(student_tau=1.2, kd_weight=0.7, ce_weight=0.3)
+    opts = K.kdkl_options(student_tau=v.student_tau, kd_weight=v.kd_weight, ce_weight=v.ce_weight,
+                          labels=torch.from_numpy(lab).cuda())
+    g = H.run_gpu(H.to_device(x), options=opts)
+    r = O.kl_loss(x.hidden_bits, x.W_bits, x.topk_idx, x.topk_logit, x.mask, x.tau, variant=v, labels=lab)
+    _parity(g, r)
