@@ -6,9 +6,10 @@
 
 One step = kdkl_forward + kdkl_backward over one batch of seeded synthetic
 inputs already resident in HBM.  Rank 0 prints one JSON line.  With N > 1
-(torchrun) every rank runs an independent replica on its own seeded batch
-(replicas only: the library is single-GPU; no collective on the data path)
-and `value` is the tokens of all ranks divided by the slowest rank's time.
+(torchrun) the step is token-sharded data parallel: every rank holds its own
+seeded batch of the workload's size (weak scaling), normalises by the
+all-reduced valid-token count and all-reduces dW over NCCL; `value` is the
+tokens of all ranks divided by the slowest rank's time.
 """
 from __future__ import annotations
 
@@ -299,10 +300,23 @@ def main_gpu(args, w: synth.Workload, N: int):
     dW = torch.empty(V, d, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    # N > 1: token-sharded data parallelism (output_head_kl_b200.dp): each rank's
+    # batch is its shard, the loss normaliser is the all-reduced valid count and
+    # dW is all-reduced (sum) over NCCL, the step's one real exchange.
+    n_total = torch.zeros(1, dtype=torch.int32, device=dev)
+    dp_opts = K.kdkl_options(n_valid_global=n_total) if world > 1 else None
+
     def step():
         K.kdkl_forward(hidden, W, idx, logit, mask, x.tau, loss, lse, ws, stream=stream)
-        K.kdkl_backward(hidden, W, idx, logit, mask, x.tau, lse, None, dH, dW, ws,
-                        chunk_tokens=args.chunk_tokens, stream=stream)
+        if world > 1:
+            n_total.copy_(ws[4:8].view(torch.int32))
+            dist.all_reduce(n_total)
+            K.kdkl_backward_ex(hidden, W, idx, logit, mask, x.tau, lse, None, dH, dW, ws, dp_opts,
+                               chunk_tokens=args.chunk_tokens, stream=stream)
+            dist.all_reduce(dW)
+        else:
+            K.kdkl_backward(hidden, W, idx, logit, mask, x.tau, lse, None, dH, dW, ws,
+                            chunk_tokens=args.chunk_tokens, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -395,7 +409,7 @@ def main_gpu(args, w: synth.Workload, N: int):
             "config": {"workload": w.name, "N": Nn, "d": d, "V": V, "K": Kc, "tau": x.tau,
                        "chunk_tokens": args.chunk_tokens or min(8192, (Nn + 127) // 128 * 128),
                        "l2": "inputs larger than L2 (W alone is %.2f GB); no flush" % (V * d * 2 / 1e9),
-                       "parallelism": f"replicas x{world}"},
+                       "parallelism": f"dp{world}" if world > 1 else "single"},
             "tflops": tflops,
             "frac_of_bf16_peak": tflops / peaks["bf16_tflops"],
             "frac_of_bf16_peak_sustained": tflops / peaks["bf16_tflops_sustained"],

@@ -176,9 +176,17 @@ typedef struct {
   int32_t kd_scale_tau_sq;  /* nonzero: multiply the KL term by student_tau^2 (default 0) */
   float ce_weight;          /* finite, >= 0 (default 0: no hard-label term) */
   const int32_t* labels;    /* [N] int32 device, 4-byte aligned; required when ce_weight > 0 */
+  /* Data-parallel normaliser: a device count to divide by instead of this
+   * call's own N_valid (e.g. the sum of every rank's kdkl_n_valid_device count
+   * after an all-reduce).  NULL = this call's own count (default). */
+  const uint32_t* n_valid_global;
 } kdkl_options;
 
 void kdkl_options_init(kdkl_options* options);
+
+/* Device address of the N_valid count that the last forward/backward on this
+ * workspace computed (uint32, stream-ordered after that call; no CUDA call is made). */
+const uint32_t* kdkl_n_valid_device(const void* workspace);
 
 /* kdkl_forward with options (NULL = defaults); topk_idx / topk_logit typed by options->cache_format. */
 kdkl_status kdkl_forward_ex(const void* hidden, const void* W, const void* topk_idx, const void* topk_logit,

@@ -38,11 +38,12 @@ CACHE_I32_F32, CACHE_U16_BF16 = 0, 1
 class Options(ctypes.Structure):
     """kdkl_options: cache format and loss-design variant (see include/kdkl.h)."""
     _fields_ = [("cache_format", ctypes.c_int32), ("student_tau", ctypes.c_float), ("kd_weight", ctypes.c_float),
-                ("kd_scale_tau_sq", ctypes.c_int32), ("ce_weight", ctypes.c_float), ("labels", ctypes.c_void_p)]
+                ("kd_scale_tau_sq", ctypes.c_int32), ("ce_weight", ctypes.c_float), ("labels", ctypes.c_void_p),
+                ("n_valid_global", ctypes.c_void_p)]
 
 
 def kdkl_options(cache_format=CACHE_I32_F32, student_tau=1.0, kd_weight=1.0, kd_scale_tau_sq=False,
-                 ce_weight=0.0, labels=None) -> Options:
+                 ce_weight=0.0, labels=None, n_valid_global=None) -> Options:
     o = Options()
     lib().kdkl_options_init(ctypes.byref(o))
     o.cache_format = int(cache_format)
@@ -51,6 +52,9 @@ def kdkl_options(cache_format=CACHE_I32_F32, student_tau=1.0, kd_weight=1.0, kd_
     o.kd_scale_tau_sq = 1 if kd_scale_tau_sq else 0
     o.ce_weight = float(ce_weight)
     o.labels = _ptr(labels)
+    o.n_valid_global = _ptr(n_valid_global)
+    # the struct holds raw device addresses: keep the tensors alive as long as it lives
+    o._keep = (labels, n_valid_global)
     return o
 
 
@@ -94,6 +98,8 @@ def lib() -> ctypes.CDLL:
     L.kdkl_teacher_topk_workspace_bytes.restype = sz
     L.kdkl_teacher_topk.argtypes = [vp, vp, i64, i32, i32, i32, vp, vp, vp, sz, vp]
     L.kdkl_teacher_topk.restype = ctypes.c_int
+    L.kdkl_n_valid_device.argtypes = [vp]
+    L.kdkl_n_valid_device.restype = ctypes.c_void_p
     L.kdkl_timing_enable.argtypes = [ctypes.c_int]
     L.kdkl_timing_enable.restype = ctypes.c_int
     L.kdkl_timing_read.argtypes = [ctypes.POINTER(KernelTime), ctypes.c_int, ctypes.c_int]
@@ -240,6 +246,11 @@ def kdkl_forward_noalloc(hidden, W, topk_idx, topk_logit, mask, tau, loss, lse, 
     if check:
         _check(st, "kdkl_forward_noalloc")
     return st
+
+
+def kdkl_n_valid_device(workspace) -> int:
+    """Device address of the workspace's N_valid count (uint32)."""
+    return int(lib().kdkl_n_valid_device(_ptr(workspace)))
 
 
 def kdkl_read_device_flags(workspace, stream=None) -> int:

@@ -195,6 +195,7 @@ kdkl_options default_options() {
   o.kd_scale_tau_sq = 0;
   o.ce_weight = 0.0f;
   o.labels = nullptr;
+  o.n_valid_global = nullptr;
   return o;
 }
 
@@ -214,6 +215,7 @@ kdkl_status check_options(const Common& c) {
     return fail(KDKL_ERR_SHAPE, "kd_weight and ce_weight must be finite and >= 0");
   if (o.ce_weight > 0.f && !o.labels) return fail(KDKL_ERR_NULL, "ce_weight > 0 needs labels");
   if (o.labels && !aligned(o.labels, 4)) return fail(KDKL_ERR_ALIGN, "labels must be 4-byte aligned");
+  if (o.n_valid_global && !aligned(o.n_valid_global, 4)) return fail(KDKL_ERR_ALIGN, "n_valid_global must be 4-byte aligned");
   return KDKL_OK;
 }
 
@@ -302,7 +304,7 @@ EpiParams base_params(const Common& c, const WsLayout& L) {
   ep.sprob = at<float>(c.ws, L.sprob);
   ep.Kp = L.Kp;
   ep.rowmask = at<uint8_t>(c.ws, L.rowmask);
-  ep.n_valid = at<uint32_t>(c.ws, L.header) + 1;
+  ep.n_valid = c.opt.n_valid_global ? c.opt.n_valid_global : at<uint32_t>(c.ws, L.header) + 1;
   ep.flags = at<uint32_t>(c.ws, L.header);
   ep.inv_tau_s = 1.0f / c.opt.student_tau;
   ep.exp_scale = 1.4426950408889634f / c.opt.student_tau;
@@ -430,7 +432,7 @@ static kdkl_status forward_impl(const void* hidden, const void* W, const void* t
          return launch_merge(ep.part_m, ep.part_s, ep.part_a, splits, pr.rows, c.opt.student_tau,
                              at<float>(workspace, L.negent), at<float>(workspace, L.wsum),
                              at<uint8_t>(workspace, L.rowmask), N, lse, loss, at<double>(workspace, L.blocksum),
-                             header, s);
+                             header, ep.n_valid, s);
        })) != cudaSuccess)
     return cuda_fail(e, "merge launch");
   return ok();
@@ -573,6 +575,10 @@ kdkl_status kdkl_backward_ex(const void* hidden, const void* W, const void* topk
 
 void kdkl_options_init(kdkl_options* options) {
   if (options) *options = default_options();
+}
+
+const uint32_t* kdkl_n_valid_device(const void* workspace) {
+  return workspace ? reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(workspace) + 4) : nullptr;
 }
 
 // ---------------------------------------------------------------- teacher top-K producer

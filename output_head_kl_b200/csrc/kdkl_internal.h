@@ -104,7 +104,7 @@ cudaError_t launch_prepass(int cache_format, const void* topk_idx, const void* t
 cudaError_t launch_merge(const float* part_m, const float* part_s, const float* part_a, int splits,
                          int rows_per_block, float student_tau, const float* negent, const float* wsum,
                          const uint8_t* rowmask, int64_t N, float* lse, float* loss, double* blocksum,
-                         uint32_t* header, cudaStream_t stream);
+                         uint32_t* header, const uint32_t* n_valid, cudaStream_t stream);
 
 // GEMM kinds: A/B majorness and epilogue are fixed per kind.
 //   kEpiLse      : A = hidden K-major, B = W K-major, BN = 256, row-stream

@@ -265,7 +265,8 @@ __global__ void __launch_bounds__(kMergeThreads)
                  const float* __restrict__ part_a, int splits, int rows_per_block, float inv_tau_s,
                  const float* __restrict__ negent, const float* __restrict__ wsum,
                  const uint8_t* __restrict__ rowmask, int64_t N, float* __restrict__ lse,
-                 float* __restrict__ loss, double* __restrict__ blocksum, uint32_t* __restrict__ header) {
+                 float* __restrict__ loss, double* __restrict__ blocksum, uint32_t* __restrict__ header,
+                 const uint32_t* __restrict__ n_valid) {
   __shared__ double s_red[kMergeThreads / 32];
   __shared__ bool s_last;
   const int64_t n = static_cast<int64_t>(blockIdx.x) * kMergeThreads + threadIdx.x;
@@ -307,7 +308,7 @@ __global__ void __launch_bounds__(kMergeThreads)
     double t = 0.0;
     const volatile double* bs = blocksum;
     for (unsigned i = 0; i < gridDim.x; ++i) t += bs[i];
-    const uint32_t nv = *reinterpret_cast<volatile uint32_t*>(&header[1]);
+    const uint32_t nv = *reinterpret_cast<const volatile uint32_t*>(n_valid);
     loss[0] = nv > 0 ? static_cast<float>(t / static_cast<double>(nv)) : 0.f;
     header[2] = 0;
   }
@@ -316,11 +317,11 @@ __global__ void __launch_bounds__(kMergeThreads)
 cudaError_t launch_merge(const float* part_m, const float* part_s, const float* part_a, int splits,
                          int rows_per_block, float student_tau, const float* negent, const float* wsum,
                          const uint8_t* rowmask, int64_t N, float* lse, float* loss, double* blocksum,
-                         uint32_t* header, cudaStream_t stream) {
+                         uint32_t* header, const uint32_t* n_valid, cudaStream_t stream) {
   const int grid = static_cast<int>((N + kMergeThreads - 1) / kMergeThreads);
   merge_kernel<<<grid, kMergeThreads, 0, stream>>>(part_m, part_s, part_a, splits, rows_per_block,
                                                    1.0f / student_tau, negent, wsum, rowmask, N, lse, loss,
-                                                   blocksum, header);
+                                                   blocksum, header, n_valid);
   return cudaGetLastError();
 }
 

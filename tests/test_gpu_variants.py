@@ -103,3 +103,21 @@ def test_variant_with_full_cache_and_label_insertion():
     g = H.run_gpu(H.to_device(x), options=opts)
     r = O.kl_loss(x.hidden_bits, x.W_bits, x.topk_idx, x.topk_logit, x.mask, x.tau, variant=v, labels=lab)
     _parity(g, r)
+
+
+def test_global_normaliser_option_and_dp_step_single_rank():
+    """n_valid_global replaces the local count (data-parallel normaliser); one rank of dp_step = plain path."""
+    from output_head_kl_b200 import dp
+    x = synth.custom_inputs(400, 128, 2000, 12, seed=308, mask_frac=0.1, w_std=0.1)
+    dx = H.to_device(x)
+    base = H.run_gpu(dx)
+    nv = int((x.mask != 0).sum())
+    doubled = torch.tensor([2 * nv], dtype=torch.int32, device="cuda")
+    g = H.run_gpu(dx, options=K.kdkl_options(n_valid_global=doubled))
+    assert g.loss == pytest.approx(base.loss / 2, rel=1e-6)
+    np.testing.assert_allclose(g.dW, base.dW / 2, rtol=1e-5, atol=1e-12)
+    res = dp.dp_step(dx.hidden, dx.W, dx.idx, dx.logit, dx.mask, dx.tau)
+    torch.cuda.synchronize()
+    assert int(res.n_valid_global.item()) == nv
+    assert res.loss.item() == pytest.approx(base.loss, rel=1e-6)
+    np.testing.assert_array_equal(res.dW.cpu().numpy(), base.dW.astype(np.float32))
