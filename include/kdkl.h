@@ -246,6 +246,18 @@ typedef struct {
 kdkl_status kdkl_timing_enable(int enable);
 int kdkl_timing_read(kdkl_kernel_time* out, int max_entries, int reset);
 
+/*
+ * Self-test of the kernels' bounded waits (failure detection without a GPU
+ * fault).  Every wait inside the kernels gives up after a time limit, sets
+ * KDKL_DEV_TIMEOUT in the workspace's flag word and lets the kernel return, so
+ * the context stays usable.  This launches one thread that waits, through the
+ * same wait routine, on a barrier that nothing completes, with a limit of
+ * limit_ns (1 us .. 1 s); afterwards kdkl_read_device_flags reports
+ * KDKL_DEV_TIMEOUT and workspace bytes [8, 16) hold the waited time (uint64 ns).
+ * workspace: >= 256 bytes, 256-byte aligned.
+ */
+kdkl_status kdkl_selftest_wait_timeout(void* workspace, uint64_t limit_ns, void* stream);
+
 /* Static name of a status code. */
 const char* kdkl_status_string(kdkl_status status);
 

@@ -100,6 +100,8 @@ def lib() -> ctypes.CDLL:
     L.kdkl_teacher_topk.restype = ctypes.c_int
     L.kdkl_n_valid_device.argtypes = [vp]
     L.kdkl_n_valid_device.restype = ctypes.c_void_p
+    L.kdkl_selftest_wait_timeout.argtypes = [vp, ctypes.c_uint64, vp]
+    L.kdkl_selftest_wait_timeout.restype = ctypes.c_int
     L.kdkl_timing_enable.argtypes = [ctypes.c_int]
     L.kdkl_timing_enable.restype = ctypes.c_int
     L.kdkl_timing_read.argtypes = [ctypes.POINTER(KernelTime), ctypes.c_int, ctypes.c_int]
@@ -258,6 +260,12 @@ def kdkl_read_device_flags(workspace, stream=None) -> int:
     _check(lib().kdkl_read_device_flags(_ptr(workspace), _stream(stream), ctypes.byref(out)),
            "kdkl_read_device_flags")
     return int(out.value)
+
+
+def kdkl_selftest_wait_timeout(workspace, limit_ns: int, stream=None) -> None:
+    """Runs the bounded-wait self-test (see include/kdkl.h); read the flags afterwards."""
+    _check(lib().kdkl_selftest_wait_timeout(_ptr(workspace), int(limit_ns), _stream(stream)),
+           "kdkl_selftest_wait_timeout")
 
 
 def kdkl_timing_enable(enable: bool = True) -> None:

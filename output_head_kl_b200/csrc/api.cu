@@ -667,6 +667,23 @@ kdkl_status kdkl_teacher_topk(const void* hidden, const void* W, int64_t N, int3
   return ok();
 }
 
+kdkl_status kdkl_selftest_wait_timeout(void* workspace, uint64_t limit_ns, void* stream) {
+  if (!workspace) return fail(KDKL_ERR_NULL, "workspace must be non-NULL");
+  if (!aligned(workspace, 256)) return fail(KDKL_ERR_ALIGN, "workspace must be 256-byte aligned");
+  if (limit_ns < 1000 || limit_ns > 1000000000ull) return fail(KDKL_ERR_SHAPE, "limit_ns outside [1 us, 1 s]");
+  Device dv;
+  kdkl_status st = current_device(dv);
+  if (st != KDKL_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, 256, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  if ((e = launch_wait_selftest(static_cast<uint32_t*>(workspace),
+                                limit_ns, reinterpret_cast<uint64_t*>(static_cast<uint8_t*>(workspace) + 8),
+                                s)) != cudaSuccess)
+    return cuda_fail(e, "self-test launch");
+  return ok();
+}
+
 kdkl_status kdkl_timing_enable(int enable) {
   std::lock_guard<std::mutex> lk(g_tmu);
   g_timing = enable != 0;

@@ -123,6 +123,9 @@ cudaError_t launch_gemm(int kind, int BN, bool pair, const CUtensorMap& tmA, con
 cudaError_t launch_topk_merge(const float* part_tv, const int* part_ti, int splits, int rows_per_block, int K,
                               int64_t N, int32_t* topk_idx, float* topk_logit, cudaStream_t stream);
 
+// Bounded-wait self-test (see kdkl_selftest_wait_timeout).
+cudaError_t launch_wait_selftest(uint32_t* flags, uint64_t limit_ns, uint64_t* waited_ns, cudaStream_t stream);
+
 // Sets the message kdkl_last_error() returns on this host thread.
 void set_last_error(const char* msg);
 

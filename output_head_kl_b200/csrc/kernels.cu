@@ -903,6 +903,31 @@ cudaError_t launch_gemm(int kind, int BN, bool pair, const CUtensorMap& tmA, con
 }
 
 // ============================================================================
+// self-test of the bounded wait: one thread waits on an mbarrier that nothing
+// completes; the wait must give up after `limit_ns`, set the timeout bit of the
+// flag word and let the kernel return normally (the context stays usable).
+// ============================================================================
+__global__ void wait_selftest_kernel(uint32_t* flags, uint64_t limit_ns, uint64_t* waited_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  abort_flag = 0;
+  fence_mbar_init();
+  AbortState ab{&abort_flag, flags};
+  ab.limit_ns = limit_ns;
+  const uint64_t t0 = globaltimer_ns();
+  const bool ok = mbar_wait(&bar, 0, ab);
+  *waited_ns = globaltimer_ns() - t0;
+  if (ok) atomicOr(flags, 0x80000000u);   // cannot happen: nothing arrives on the barrier
+}
+
+cudaError_t launch_wait_selftest(uint32_t* flags, uint64_t limit_ns, uint64_t* waited_ns, cudaStream_t stream) {
+  wait_selftest_kernel<<<1, 32, 0, stream>>>(flags, limit_ns, waited_ns);
+  return cudaGetLastError();
+}
+
+// ============================================================================
 // top-K merge: one warp per row sorts the row's split heaps (bitonic, in
 // shared memory) by (value descending, index ascending) and keeps the first K
 // ============================================================================

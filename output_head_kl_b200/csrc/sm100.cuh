@@ -59,6 +59,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 struct AbortState {
   volatile int* smem_flag;   // set to 1 by the first role that gives up
   uint32_t* gmem_flags;      // device flag word (KDKL_DEV_* bits)
+  uint64_t limit_ns = kWaitLimitNs;
 };
 
 // Waits for the phase with `parity` to complete.  Returns false if the wait
@@ -72,7 +73,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(a, parity)) return true;
     if (*ab.smem_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > ab.limit_ns) {
       *ab.smem_flag = 1;
       atomicOr(ab.gmem_flags, kFlagTimeout);
       return false;
