@@ -179,6 +179,38 @@ def gpu_id_for(dev_index: int) -> str:
     return str(dev_index)
 
 
+# ----------------------------------------------------------------------------- same-box reference
+def same_box_gemm_reference(dev, seconds: float = 3.0, size: int = 8192):
+    """cuBLAS bf16 GEMM (torch.matmul, 2 n^3 flops) looped for `seconds` on this GPU,
+    with its clock: context for how much of the gap to the fixed peak is this box's
+    power-capped clock.  Not a kernel of this library."""
+    import torch
+    a = torch.randn(size, size, device=dev, dtype=torch.bfloat16)
+    b = torch.randn(size, size, device=dev, dtype=torch.bfloat16)
+    c = torch.empty(size, size, device=dev, dtype=torch.bfloat16)
+    for _ in range(3):
+        torch.matmul(a, b, out=c)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.perf_counter()
+    sampler = ClockSampler(gpu_id_for(dev.index or 0))
+    sampler.start()
+    n = 0
+    e0.record()
+    while time.perf_counter() - t0 < seconds:
+        for _ in range(10):
+            torch.matmul(a, b, out=c)
+        n += 10
+        torch.cuda.synchronize()
+    e1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1) / n
+    del a, b, c
+    return {"kind": "cuBLAS bf16 GEMM 8192^3 via torch.matmul, sustained loop", "tflops": 2.0 * size ** 3 / ms / 1e9,
+            "sm_mhz": clocks.get("sm_mhz"), "reasons": clocks.get("reasons")}
+
+
 # ----------------------------------------------------------------------------- oracle arm
 def oracle_sample(x: synth.Inputs, rows: int, seed: int):
     """Times the CPU oracle (as it stands) on a bounded sample of the workload's rows."""
@@ -373,6 +405,9 @@ def main_gpu(args, w: synth.Workload, N: int):
     d2h = 4
 
     out = None
+    ref_gemm = None
+    if rank == 0 and not args.no_gemm_reference:
+        ref_gemm = same_box_gemm_reference(dev)
     if rank == 0:
         peaks = measured_peaks()
         flops = synth.flops_fwd_bwd(Nn, d, V)
@@ -413,6 +448,8 @@ def main_gpu(args, w: synth.Workload, N: int):
             "tflops": tflops,
             "frac_of_bf16_peak": tflops / peaks["bf16_tflops"],
             "frac_of_bf16_peak_sustained": tflops / peaks["bf16_tflops_sustained"],
+            "same_box_cublas": ref_gemm,
+            "frac_of_same_box_cublas": (tflops / ref_gemm["tflops"]) if ref_gemm else None,
             "peak_gb": peak_bytes / 1e9,
             "workspace_gb": ws_bytes / 1e9,
             "roofline": roof,
@@ -495,6 +532,8 @@ def main():
     ap.add_argument("--N", type=int, default=None, help="token count override (sweep points)")
     ap.add_argument("--chunk-tokens", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-gemm-reference", action="store_true",
+                    help="skip the same-box cuBLAS GEMM timed after the run (context only)")
     ap.add_argument("--topk", action="store_true", help="time the teacher top-K cache producer instead")
     ap.add_argument("--record-traffic", metavar="NCU_CSV",
                     help="write profiles/traffic.json from an ncu dram__bytes capture of --config's workload")
@@ -512,6 +551,7 @@ def main():
         return main_topk(args, w, N)
     if args.sweep:
         args.no_cpu_baseline = True
+        args.no_gemm_reference = True
         for n in synth.SWEEP_N:
             rc = main_gpu(args, synth.CONFIGS["sweep"], n)
             if rc:
