@@ -179,10 +179,10 @@ def gpu_id_for(dev_index: int) -> str:
     return str(dev_index)
 
 
-# ----------------------------------------------------------------------------- same-box reference
-def same_box_gemm_reference(dev, seconds: float = 3.0, size: int = 8192):
+# ----------------------------------------------------------------------------- same-GPU reference
+def same_gpu_gemm_reference(dev, seconds: float = 3.0, size: int = 8192):
     """cuBLAS bf16 GEMM (torch.matmul, 2 n^3 flops) looped for `seconds` on this GPU,
-    with its clock: context for how much of the gap to the fixed peak is this box's
+    with its clock: context for how much of the gap to the fixed peak is this GPU's
     power-capped clock.  Not a kernel of this library."""
     import torch
     a = torch.randn(size, size, device=dev, dtype=torch.bfloat16)
@@ -407,7 +407,7 @@ def main_gpu(args, w: synth.Workload, N: int):
     out = None
     ref_gemm = None
     if rank == 0 and not args.no_gemm_reference:
-        ref_gemm = same_box_gemm_reference(dev)
+        ref_gemm = same_gpu_gemm_reference(dev)
     if rank == 0:
         peaks = measured_peaks()
         flops = synth.flops_fwd_bwd(Nn, d, V)
@@ -448,8 +448,8 @@ def main_gpu(args, w: synth.Workload, N: int):
             "tflops": tflops,
             "frac_of_bf16_peak": tflops / peaks["bf16_tflops"],
             "frac_of_bf16_peak_sustained": tflops / peaks["bf16_tflops_sustained"],
-            "same_box_cublas": ref_gemm,
-            "frac_of_same_box_cublas": (tflops / ref_gemm["tflops"]) if ref_gemm else None,
+            "same_gpu_cublas": ref_gemm,
+            "frac_of_same_gpu_cublas": (tflops / ref_gemm["tflops"]) if ref_gemm else None,
             "peak_gb": peak_bytes / 1e9,
             "workspace_gb": ws_bytes / 1e9,
             "roofline": roof,
@@ -533,7 +533,7 @@ def main():
     ap.add_argument("--chunk-tokens", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-gemm-reference", action="store_true",
-                    help="skip the same-box cuBLAS GEMM timed after the run (context only)")
+                    help="skip the same-GPU cuBLAS GEMM timed after the run (context only)")
     ap.add_argument("--topk", action="store_true", help="time the teacher top-K cache producer instead")
     ap.add_argument("--record-traffic", metavar="NCU_CSV",
                     help="write profiles/traffic.json from an ncu dram__bytes capture of --config's workload")
