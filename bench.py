@@ -338,16 +338,17 @@ def main_gpu(args, w: synth.Workload, N: int):
     n_total = torch.zeros(1, dtype=torch.int32, device=dev)
     dp_opts = K.kdkl_options(n_valid_global=n_total) if world > 1 else None
 
-    def step():
-        K.kdkl_forward(hidden, W, idx, logit, mask, x.tau, loss, lse, ws, stream=stream)
+    def step(bufs=None):
+        hidden_, idx_, logit_, mask_ = bufs if bufs is not None else (hidden, idx, logit, mask)
+        K.kdkl_forward(hidden_, W, idx_, logit_, mask_, x.tau, loss, lse, ws, stream=stream)
         if world > 1:
             n_total.copy_(ws[4:8].view(torch.int32))
             dist.all_reduce(n_total)
-            K.kdkl_backward_ex(hidden, W, idx, logit, mask, x.tau, lse, None, dH, dW, ws, dp_opts,
+            K.kdkl_backward_ex(hidden_, W, idx_, logit_, mask_, x.tau, lse, None, dH, dW, ws, dp_opts,
                                chunk_tokens=args.chunk_tokens, stream=stream)
             dist.all_reduce(dW)
         else:
-            K.kdkl_backward(hidden, W, idx, logit, mask, x.tau, lse, None, dH, dW, ws,
+            K.kdkl_backward(hidden_, W, idx_, logit_, mask_, x.tau, lse, None, dH, dW, ws,
                             chunk_tokens=args.chunk_tokens, stream=stream)
 
     for _ in range(args.warmup):
@@ -380,27 +381,47 @@ def main_gpu(args, w: synth.Workload, N: int):
     ms = e0.elapsed_time(e1) / args.steps
     ms_max = max_over_ranks(ms, dev, world)
 
-    # end-to-end through the public API with host buffers: per step the batch
-    # (hidden, cache, mask) goes host -> device from pinned memory and the
-    # loss comes back device -> host
+    # end-to-end through the public API with host buffers: every step's batch
+    # (hidden, cache, mask) goes host -> device from pinned memory and its loss
+    # comes back device -> host.  As a data loader would, the next batch's copy
+    # runs on a second stream into a second set of buffers while this step
+    # computes (the copy of batch i+1 waits until step i-1 has released them).
     h_loss = torch.empty(1, dtype=torch.float32).pin_memory()
     e2e_steps = args.steps
+    bufs = [(hidden, idx, logit, mask),
+            (torch.empty_like(hidden), torch.empty_like(idx), torch.empty_like(logit), torch.empty_like(mask))]
+    copy_stream = torch.cuda.Stream(dev)
+    copied = [torch.cuda.Event(), torch.cuda.Event()]
+    released = [torch.cuda.Event(), torch.cuda.Event()]
+
+    def fetch(i):
+        b = bufs[i % 2]
+        with torch.cuda.stream(copy_stream):
+            if i >= 2:
+                copy_stream.wait_event(released[i % 2])
+            for dst, src in zip(b, (h_hidden, h_idx, h_logit, h_mask)):
+                dst.copy_(src, non_blocking=True)
+            copied[i % 2].record(copy_stream)
+
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
-    for _ in range(e2e_steps):
-        hidden.copy_(h_hidden, non_blocking=True)
-        idx.copy_(h_idx, non_blocking=True)
-        logit.copy_(h_logit, non_blocking=True)
-        mask.copy_(h_mask, non_blocking=True)
-        step()
+    copy_stream.wait_event(t0)
+    fetch(0)
+    for i in range(e2e_steps):
+        if i + 1 < e2e_steps:
+            fetch(i + 1)
+        stream.wait_event(copied[i % 2])
+        step(bufs[i % 2])
+        released[i % 2].record(stream)
         h_loss.copy_(loss, non_blocking=True)
     t1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(t0.elapsed_time(t1) / e2e_steps, dev, world)
+    del bufs
     h2d = Nn * d * 2 + Nn * Kc * 4 * 2 + Nn
     d2h = 4
 
