@@ -300,7 +300,7 @@ def main_gpu(args, w: synth.Workload, N: int):
     dev = torch.device("cuda", local)
     if world > 1:
         import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=dev)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
 
     K.lib()
     t_gen = time.perf_counter()
@@ -319,6 +319,8 @@ def main_gpu(args, w: synth.Workload, N: int):
     torch.cuda.reset_peak_memory_stats(dev)
     base_alloc = torch.cuda.memory_allocated(dev)
     W = bf16(x.W_bits).to(dev)
+    if world > 1:
+        dist.broadcast(W, src=0)     # one output-head weight, replicated (data parallelism)
 
     hidden = h_hidden.to(dev)
     idx = h_idx.to(dev)
