@@ -460,12 +460,13 @@ def main_gpu(args, w: synth.Workload, N: int):
             cpu = {"value": n_rows / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                    "sample": f"{n_rows} seeded rows of the {w.name} workload, one full fwd+bwd "
                              f"(loss, lse, dHidden, dW contribution) in numpy float64, {dt:.1f} s"}
+        bwd_plan = K.kdkl_backward_plan(Nn, d, V, Kc, args.chunk_tokens)
         out = {
             "metric": METRIC, "value": Nn * world / (ms_max * 1e-3), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "N": Nn, "d": d, "V": V, "K": Kc, "tau": x.tau,
-                       "chunk_tokens": args.chunk_tokens or min(8192, (Nn + 127) // 128 * 128),
+                       "chunk_tokens": bwd_plan[1], "bwd_tile_n": bwd_plan[0],
                        "l2": "inputs larger than L2 (W alone is %.2f GB); no flush" % (V * d * 2 / 1e9),
                        "parallelism": f"dp{world}" if world > 1 else "single"},
             "tflops": tflops,

@@ -180,6 +180,12 @@ typedef struct {
    * call's own N_valid (e.g. the sum of every rank's kdkl_n_valid_device count
    * after an all-reduce).  NULL = this call's own count (default). */
   const uint32_t* n_valid_global;
+  /* N tile width of the backward's dHidden and dW GEMMs (their N axis is d):
+   * 0 = the planner's choice (default; see kdkl_backward_plan), else one of
+   * 128, 160, 192, 224, 240, 256.  It changes how the output is partitioned
+   * into tiles, not the arithmetic: each output element is accumulated over
+   * the same 64-wide reduction blocks in the same order. */
+  int32_t bwd_tile_n;
 } kdkl_options;
 
 void kdkl_options_init(kdkl_options* options);
@@ -193,6 +199,24 @@ kdkl_status kdkl_forward_ex(const void* hidden, const void* W, const void* topk_
                             const uint8_t* mask, int64_t N, int32_t d, int32_t V, int32_t K, float tau,
                             const kdkl_options* options, float* loss, float* lse, void* workspace,
                             size_t workspace_bytes, void* stream);
+
+/*
+ * The backward's work plan, computed on the host without any CUDA work: the N
+ * tile width of the dHidden and dW GEMMs and the tokens per chunk that
+ * kdkl_backward / kdkl_backward_ex use for these arguments on a device with
+ * `sm_count` SMs (0 = ask the current device).  An explicit chunk_tokens is
+ * used as given (rounded up to a multiple of 128, at most N rounded up); with
+ * chunk_tokens = 0 the chunk is chosen at or below the workspace's default
+ * chunk capacity (8192 tokens).  The planner minimises a wave-count cost model
+ * of the two GEMMs: the dHidden GEMM has only (chunk / 256) x ceil(d / tile_n)
+ * output tiles, each reducing over the whole vocabulary, so a partly filled
+ * last wave of tiles idles most of the GPU for a long time.
+ * Errors: KDKL_ERR_NULL (an output pointer is NULL), KDKL_ERR_SHAPE,
+ * KDKL_ERR_UNSUPPORTED (bad options or no device when sm_count = 0).
+ */
+kdkl_status kdkl_backward_plan(int64_t N, int32_t d, int32_t V, int32_t K, int64_t chunk_tokens,
+                               const kdkl_options* options, int32_t sm_count, int32_t* tile_n_out,
+                               int64_t* chunk_tokens_out);
 
 /* kdkl_backward with options (NULL = defaults); must match the forward's options. */
 kdkl_status kdkl_backward_ex(const void* hidden, const void* W, const void* topk_idx, const void* topk_logit,
@@ -210,7 +234,7 @@ kdkl_status kdkl_backward_ex(const void* hidden, const void* W, const void* topk
  * output head, this computes z = hidden W^T tile by tile on the tensor cores
  * (never storing z) and keeps each row's K largest logits:
  *   hidden      [N, d] bf16, 16-byte aligned; W [V, d] bf16, 16-byte aligned
- *   1 <= K <= 128, K <= V, d % 8 == 0
+ *   1 <= K <= 128, K <= V <= 65,280 * floor(1024 / K) (522,240 at K = 128), d % 8 == 0
  *   topk_idx    [N, K] int32 out; topk_logit [N, K] fp32 out (the fp32 logits z)
  *   each row ordered by logit descending, ties to the smaller index
  *   workspace   >= kdkl_teacher_topk_workspace_bytes(N, d, V, K), 256-byte aligned

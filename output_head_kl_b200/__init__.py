@@ -39,11 +39,11 @@ class Options(ctypes.Structure):
     """kdkl_options: cache format and loss-design variant (see include/kdkl.h)."""
     _fields_ = [("cache_format", ctypes.c_int32), ("student_tau", ctypes.c_float), ("kd_weight", ctypes.c_float),
                 ("kd_scale_tau_sq", ctypes.c_int32), ("ce_weight", ctypes.c_float), ("labels", ctypes.c_void_p),
-                ("n_valid_global", ctypes.c_void_p)]
+                ("n_valid_global", ctypes.c_void_p), ("bwd_tile_n", ctypes.c_int32)]
 
 
 def kdkl_options(cache_format=CACHE_I32_F32, student_tau=1.0, kd_weight=1.0, kd_scale_tau_sq=False,
-                 ce_weight=0.0, labels=None, n_valid_global=None) -> Options:
+                 ce_weight=0.0, labels=None, n_valid_global=None, bwd_tile_n=0) -> Options:
     o = Options()
     lib().kdkl_options_init(ctypes.byref(o))
     o.cache_format = int(cache_format)
@@ -53,6 +53,7 @@ def kdkl_options(cache_format=CACHE_I32_F32, student_tau=1.0, kd_weight=1.0, kd_
     o.ce_weight = float(ce_weight)
     o.labels = _ptr(labels)
     o.n_valid_global = _ptr(n_valid_global)
+    o.bwd_tile_n = int(bwd_tile_n)
     # the struct holds raw device addresses: keep the tensors alive as long as it lives
     o._keep = (labels, n_valid_global)
     return o
@@ -106,6 +107,9 @@ def lib() -> ctypes.CDLL:
     L.kdkl_timing_enable.restype = ctypes.c_int
     L.kdkl_timing_read.argtypes = [ctypes.POINTER(KernelTime), ctypes.c_int, ctypes.c_int]
     L.kdkl_timing_read.restype = ctypes.c_int
+    L.kdkl_backward_plan.argtypes = [i64, i32, i32, i32, i64, ctypes.POINTER(Options), i32,
+                                     ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int64)]
+    L.kdkl_backward_plan.restype = ctypes.c_int
     _lib = L
     return L
 
@@ -142,6 +146,18 @@ def kdkl_last_error() -> str:
 
 def kdkl_workspace_bytes(N: int, d: int, V: int, K: int, chunk_tokens: int = 0) -> int:
     return int(lib().kdkl_workspace_bytes(N, d, V, K, chunk_tokens))
+
+
+def kdkl_backward_plan(N: int, d: int, V: int, K: int, chunk_tokens: int = 0, options: Options | None = None,
+                       sm_count: int = 0) -> tuple[int, int]:
+    """(tile_n, chunk_tokens) the backward uses for these sizes; sm_count 0 = the current device."""
+    tn = ctypes.c_int32()
+    ch = ctypes.c_int64()
+    st = lib().kdkl_backward_plan(int(N), int(d), int(V), int(K), int(chunk_tokens),
+                                  ctypes.byref(options) if options is not None else None, int(sm_count),
+                                  ctypes.byref(tn), ctypes.byref(ch))
+    _check(st, "kdkl_backward_plan")
+    return tn.value, ch.value
 
 
 def kdkl_forward(hidden, W, topk_idx, topk_logit, mask, tau, loss, lse, workspace, *, N=None, d=None, V=None,

@@ -99,12 +99,13 @@ kdkl_status current_device(Device& dv) {
 // vocabulary tiles: balance the per-group tile count over `ctas` CTA groups
 // (single CTAs or CTA pairs), and keep at least enough splits that the hidden
 // rows in flight stay small next to L2.  `units_cap` bounds rb * splits.
-int pick_splits(int64_t rb, int vt, int ctas, int d, int64_t units_cap, int rows_per_block) {
+int pick_splits(int64_t rb, int vt, int ctas, int d, int64_t units_cap, int rows_per_block, int s_floor = 1) {
   // Measured on the 8B-class head: the forward is fastest with about 9
   // 256-row blocks (18 MB of hidden rows) in flight; 37 MB already thrashes L2.
   const double rows_bytes = static_cast<double>(rows_per_block) * d * 2.0;
   const double budget = 20.0 * 1024 * 1024;
   int s_min = static_cast<int>(std::ceil(ctas * rows_bytes / budget));
+  if (s_min < s_floor) s_min = s_floor;
   if (s_min < 1) s_min = 1;
   int s_max = static_cast<int>(units_cap / rb);
   if (s_max > vt) s_max = vt;
@@ -126,12 +127,18 @@ int pick_splits(int64_t rb, int vt, int ctas, int d, int64_t units_cap, int rows
   return s_min;
 }
 
-// Tile width of the dHidden / dW GEMMs (their N dimension is d).  256-wide
-// tiles run as CTA pairs (cta_group::2), which keep the tensor pipe about 15
-// points busier per clock than single-CTA tiles, so they win unless padding d
-// up to a multiple of 256 wastes more than 1/8 of the work; then the
-// narrower single-CTA tile with the least padding is used.
-int pick_bn(int d) {
+// Tile widths (N, over d) of the dHidden / dW GEMMs.  CTA pairs (cta_group::2,
+// 256-row tiles) run any width in kPairTileN; single CTAs, used only on a
+// device with one SM, run 256, 192 or 128.
+constexpr int kPairTileN[] = {256, 240, 224, 192, 160, 128};
+
+bool pair_tile_n_ok(int bn) {
+  for (int t : kPairTileN)
+    if (t == bn) return true;
+  return false;
+}
+
+int pick_bn_single(int d) {
   const int64_t pad256 = static_cast<int64_t>((d + 255) / 256) * 256;
   const int64_t pad192 = static_cast<int64_t>((d + 191) / 192) * 192;
   const int64_t pad128 = static_cast<int64_t>((d + 127) / 128) * 128;
@@ -141,7 +148,7 @@ int pick_bn(int d) {
 }
 
 // Whether a GEMM runs as CTA pairs (256-row tiles, cta_group::2) or single
-// CTAs (128-row tiles).  Pairs need the 256-wide N tile (split 128 + 128).
+// CTAs (128-row tiles).
 struct Pairing {
   bool pair;
   int rows;     // rows of one tile / unit
@@ -153,13 +160,109 @@ struct Pairing {
   }
 };
 
-Pairing pairing(const Device& dv, int bn) {
+Pairing pairing(int sms, int bn) {
   Pairing p;
-  p.pair = (bn == 256) && dv.sms >= 2;
+  p.pair = sms >= 2;
   p.rows = p.pair ? 2 * kBM : kBM;
-  p.groups = p.pair ? dv.sms / 2 : dv.sms;
+  p.groups = p.pair ? sms / 2 : sms;
   p.b_rows = p.pair ? bn / 2 : bn;
   return p;
+}
+
+// Backward plan: tile width of the dHidden / dW GEMMs and tokens per chunk.
+//
+// Cost model (seconds, at an assumed kPlanSmRate flop/s per SM): per chunk of
+// nc tokens, the dHidden GEMM runs ceil(ceil(nc / rows) * nt / groups) waves of
+// tiles that each reduce over the whole vocabulary (2 * rows * bn * V flops),
+// and the dW GEMM ceil(ceil(V / rows) * nt / groups) waves of tiles reducing
+// over the chunk (2 * rows * bn * nc flops); a tile of width bn runs at
+// tile_efficiency(bn) of the 256-wide tile's flop rate, every tile adds
+// kPlanTileFixed and every chunk kPlanChunkFixed.  With V in the hundreds of
+// thousands a dHidden tile runs for about a millisecond, so a partly filled
+// last wave costs more than an extra chunk.  Among plans within 1 % of the
+// cheapest, the widest tile and then the largest chunk win.
+constexpr double kPlanSmRate = 8.0e12;
+constexpr double kPlanTileFixed = 2.0e-6;
+constexpr double kPlanChunkFixed = 40.0e-6;
+
+// Flop rate of a CTA-pair tile of width bn relative to the 256-wide tile, as
+// measured on B200 from the dHidden and dW kernels' times at equal work, scaled
+// by the sampled SM clock (d = 2880, 3584 and 4096): narrower tiles stream the
+// same A operand for fewer MMA flops and turn their pipeline stages over faster.
+double tile_efficiency(int bn) {
+  switch (bn) {
+    case 256: return 1.0;
+    case 240: return 0.87;
+    case 224: return 0.92;
+    case 192: return 0.75;
+    case 160: return 0.67;
+    default: return 0.5;
+  }
+}
+
+double backward_cost(int64_t N, int d, int V, int bn, int64_t chunk, const Pairing& p) {
+  const double rate = kPlanSmRate * (p.pair ? 2.0 : 1.0) * tile_efficiency(bn);
+  const int64_t nt = (d + bn - 1) / bn;
+  const int64_t vb = (V + p.rows - 1) / p.rows;
+  auto chunk_cost = [&](int64_t nc) {
+    const int64_t rb = (nc + p.rows - 1) / p.rows;
+    const int64_t w_dh = (rb * nt + p.groups - 1) / p.groups;
+    const int64_t w_dw = (vb * nt + p.groups - 1) / p.groups;
+    const double t_dh = 2.0 * p.rows * bn * static_cast<double>(V) / rate + kPlanTileFixed;
+    const double t_dw = 2.0 * p.rows * bn * static_cast<double>(nc) / rate + kPlanTileFixed;
+    return static_cast<double>(w_dh) * t_dh + static_cast<double>(w_dw) * t_dw + kPlanChunkFixed;
+  };
+  const int64_t full = N / chunk, rest = N % chunk;
+  return static_cast<double>(full) * chunk_cost(chunk) + (rest ? chunk_cost(rest) : 0.0);
+}
+
+struct BackwardPlan {
+  int bn;
+  int64_t chunk;
+};
+
+// `cap` = the workspace's chunk capacity (L.chunk); `auto_chunk` = chunk_tokens was 0.
+BackwardPlan plan_backward(int64_t N, int d, int V, int64_t cap, bool auto_chunk, int forced_bn, int sms) {
+  BackwardPlan best{256, cap};
+  if (sms < 2) {
+    best.bn = pick_bn_single(d);
+    return best;
+  }
+  const Pairing p = pairing(sms, 256);
+  struct Cand {
+    double cost;
+    int bn;
+    int64_t chunk;
+  };
+  Cand cands[6 * 64];
+  int n = 0;
+  double lo = 1e300;
+  for (int bn : kPairTileN) {
+    if (forced_bn && bn != forced_bn) continue;
+    // chunk candidates: the capacity itself, then multiples of the tile height below it
+    int64_t ch = cap;
+    int taken = 0;
+    while (ch >= 1 && taken < 64) {
+      const double cost = backward_cost(N, d, V, bn, ch, p);
+      cands[n++] = Cand{cost, bn, ch};
+      lo = cost < lo ? cost : lo;
+      ++taken;
+      if (!auto_chunk) break;
+      const int64_t next = (ch - 1) / p.rows * p.rows;
+      if (next < p.rows) break;
+      ch = next;
+    }
+  }
+  bool have = false;
+  for (int i = 0; i < n; ++i) {
+    if (cands[i].cost > lo * 1.01) continue;
+    if (!have || cands[i].bn > best.bn || (cands[i].bn == best.bn && cands[i].chunk > best.chunk)) {
+      best.bn = cands[i].bn;
+      best.chunk = cands[i].chunk;
+      have = true;
+    }
+  }
+  return best;
 }
 
 kdkl_status check_shapes(int64_t N, int32_t d, int32_t V, int32_t K, float tau) {
@@ -196,6 +299,7 @@ kdkl_options default_options() {
   o.ce_weight = 0.0f;
   o.labels = nullptr;
   o.n_valid_global = nullptr;
+  o.bwd_tile_n = 0;
   return o;
 }
 
@@ -216,6 +320,8 @@ kdkl_status check_options(const Common& c) {
   if (o.ce_weight > 0.f && !o.labels) return fail(KDKL_ERR_NULL, "ce_weight > 0 needs labels");
   if (o.labels && !aligned(o.labels, 4)) return fail(KDKL_ERR_ALIGN, "labels must be 4-byte aligned");
   if (o.n_valid_global && !aligned(o.n_valid_global, 4)) return fail(KDKL_ERR_ALIGN, "n_valid_global must be 4-byte aligned");
+  if (o.bwd_tile_n != 0 && !pair_tile_n_ok(o.bwd_tile_n))
+    return fail(KDKL_ERR_UNSUPPORTED, "bwd_tile_n=%d is not 0 or one of 128, 160, 192, 224, 240, 256", o.bwd_tile_n);
   return KDKL_OK;
 }
 
@@ -400,7 +506,7 @@ static kdkl_status forward_impl(const void* hidden, const void* W, const void* t
   }
   if ((st = run_prepass(c, L, s)) != KDKL_OK) return st;
 
-  const Pairing pr = pairing(dv, 256);
+  const Pairing pr = pairing(dv.sms, 256);
   const int64_t rb = (N + pr.rows - 1) / pr.rows;
   const int vt = (V + 255) / 256;
   const int splits = pick_splits(rb, vt, pr.groups, d, L.units_cap * kBM / pr.rows, pr.rows);
@@ -480,9 +586,11 @@ static kdkl_status backward_impl(const void* hidden, const void* W, const void* 
   if ((st = run_prepass(c, L, s)) != KDKL_OK) return st;
 
   uint16_t* gbuf = at<uint16_t>(workspace, L.gbuf);
-  const Pairing pg = pairing(dv, 256);          // logit recompute (always 256-wide vocabulary tiles)
-  const int bn = pick_bn(d);
-  const Pairing pd = pairing(dv, bn);           // dHidden and dW GEMMs
+  const Pairing pg = pairing(dv.sms, 256);          // logit recompute (always 256-wide vocabulary tiles)
+  const BackwardPlan plan = plan_backward(N, d, V, L.chunk, chunk_tokens == 0, c.opt.bwd_tile_n, dv.sms);
+  const int bn = plan.bn;
+  const int64_t chunk = plan.chunk;
+  const Pairing pd = pairing(dv.sms, bn);       // dHidden and dW GEMMs
   CUtensorMap tmW_k;  // W as K-major B of the logit recompute
   CUtensorMap tmW_mn; // W as MN-major B of dHidden = G W
   if (!make_map(&tmW_k, W, d, V, d, kBK, pg.b_rows, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -494,8 +602,8 @@ static kdkl_status backward_impl(const void* hidden, const void* W, const void* 
   ep0.lse = lse;
   ep0.grad_loss = grad_loss;
 
-  for (int64_t c0 = 0; c0 < N; c0 += L.chunk) {
-    const int64_t nc = (N - c0) < L.chunk ? (N - c0) : L.chunk;
+  for (int64_t c0 = 0; c0 < N; c0 += chunk) {
+    const int64_t nc = (N - c0) < chunk ? (N - c0) : chunk;
     const void* hc = static_cast<const uint8_t*>(hidden) + static_cast<size_t>(c0) * d * 2;
     CUtensorMap tmH_k, tmH_mn, tmG_store, tmG_k, tmG_mn;
     if (!make_map(&tmH_k, hc, d, nc, d, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -577,6 +685,30 @@ void kdkl_options_init(kdkl_options* options) {
   if (options) *options = default_options();
 }
 
+kdkl_status kdkl_backward_plan(int64_t N, int32_t d, int32_t V, int32_t K, int64_t chunk_tokens,
+                               const kdkl_options* options, int32_t sm_count, int32_t* tile_n_out,
+                               int64_t* chunk_tokens_out) {
+  if (!tile_n_out || !chunk_tokens_out) return fail(KDKL_ERR_NULL, "tile_n_out and chunk_tokens_out must be non-NULL");
+  kdkl_status st = check_shapes(N, d, V, K, 1.0f);
+  if (st != KDKL_OK) return st;
+  if (chunk_tokens < 0) return fail(KDKL_ERR_SHAPE, "chunk_tokens must be >= 0");
+  if (sm_count < 0) return fail(KDKL_ERR_SHAPE, "sm_count must be >= 0");
+  const kdkl_options o = options ? *options : default_options();
+  if (o.bwd_tile_n != 0 && !pair_tile_n_ok(o.bwd_tile_n))
+    return fail(KDKL_ERR_UNSUPPORTED, "bwd_tile_n=%d is not 0 or one of 128, 160, 192, 224, 240, 256", o.bwd_tile_n);
+  int sms = sm_count;
+  if (sms == 0) {
+    Device dv;
+    if ((st = current_device(dv)) != KDKL_OK) return st;
+    sms = dv.sms;
+  }
+  const WsLayout L = make_layout(N, d, V, K, chunk_tokens);
+  const BackwardPlan plan = plan_backward(N, d, V, L.chunk, chunk_tokens == 0, o.bwd_tile_n, sms);
+  *tile_n_out = plan.bn;
+  *chunk_tokens_out = plan.chunk;
+  return ok();
+}
+
 const uint32_t* kdkl_n_valid_device(const void* workspace) {
   return workspace ? reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(workspace) + 4) : nullptr;
 }
@@ -590,7 +722,7 @@ struct TopkLayout {
 
 TopkLayout topk_layout(int64_t N, int32_t K) {
   TopkLayout L;
-  L.s_cap = 1024 / K > 0 ? 1024 / K : 1;
+  L.s_cap = kTopKMergeCand / K > 0 ? kTopKMergeCand / K : 1;
   // enough partial slots for either tile height (256-row pairs or 128-row CTAs)
   const size_t slots = static_cast<size_t>((N + 255) / 256 + 1) * 256 * L.s_cap * K;
   size_t off = 256;
@@ -607,6 +739,12 @@ kdkl_status check_topk_shapes(int64_t N, int32_t d, int32_t V, int32_t K) {
   if (d < 8 || d % 8 != 0) return fail(KDKL_ERR_SHAPE, "d=%d must be a positive multiple of 8", d);
   if (V < 1 || V > kMaxV) return fail(KDKL_ERR_SHAPE, "V=%d outside [1, 2^30]", V);
   if (K < 1 || K > kTopKMax || K > V) return fail(KDKL_ERR_SHAPE, "K=%d outside [1, min(%d, V)]", K, kTopKMax);
+  // every vocabulary split spans at most kTopKUnitTiles tiles, with at most
+  // kTopKMergeCand / K splits
+  const int64_t vt = (static_cast<int64_t>(V) + 255) / 256;
+  const int64_t s_cap = kTopKMergeCand / K;
+  if ((vt + s_cap - 1) / s_cap > kTopKUnitTiles)
+    return fail(KDKL_ERR_SHAPE, "V=%d above %lld for K=%d", V, (long long)(kTopKUnitTiles * 256LL * s_cap), K);
   return KDKL_OK;
 }
 }  // namespace
@@ -632,7 +770,7 @@ kdkl_status kdkl_teacher_topk(const void* hidden, const void* W, int64_t N, int3
     return fail(KDKL_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, L.total);
   Device dv;
   if ((st = current_device(dv)) != KDKL_OK) return st;
-  const Pairing pr = pairing(dv, 256);
+  const Pairing pr = pairing(dv.sms, 256);
   if (!pr.pair) return fail(KDKL_ERR_UNSUPPORTED, "the top-K producer needs CTA pairs");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
@@ -640,7 +778,8 @@ kdkl_status kdkl_teacher_topk(const void* hidden, const void* W, int64_t N, int3
   if (N == 0) return ok();
   const int64_t rb = (N + pr.rows - 1) / pr.rows;
   const int vt = (V + 255) / 256;
-  const int splits = pick_splits(rb, vt, pr.groups, d, rb * L.s_cap, pr.rows);
+  const int splits = pick_splits(rb, vt, pr.groups, d, rb * L.s_cap, pr.rows,
+                                 (vt + kTopKUnitTiles - 1) / kTopKUnitTiles);
   Sched sc{static_cast<int>(rb * splits), splits, vt, (d + kBK - 1) / kBK, 1};
   CUtensorMap tmA, tmB;
   if (!make_map(&tmA, hidden, d, N, d, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||

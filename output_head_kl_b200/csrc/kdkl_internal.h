@@ -91,8 +91,15 @@ struct EpiParams {
 enum EpiKind { kEpiLse = 0, kEpiGrad = 1, kEpiStoreBf16 = 2, kEpiRmwF32 = 3, kEpiTopK = 4 };
 
 // Teacher top-K producer: per-row min-heaps of up to kTopKMax entries live in
-// shared memory during the vocabulary sweep.
+// shared memory during the vocabulary sweep, with 16-bit indices relative to
+// the unit's first column; a unit therefore spans at most kTopKUnitTiles
+// 256-column tiles (the planner's vocabulary splits guarantee it), and
+// kTopKEmpty (above every relative index) marks an empty heap slot.
 constexpr int kTopKMax = 128;
+constexpr int kTopKUnitTiles = 255;
+constexpr int kTopKEmpty = 0xFFFF;
+// Per-row candidates the top-K merge sorts (vocabulary splits x K).
+constexpr int kTopKMergeCand = 1024;
 
 // Launchers (defined in kernels.cu).  Each returns cudaGetLastError() of its launch.
 // cache_format 0: int32 indices + fp32 logits; 1: uint16 indices + bf16 logits.

@@ -343,22 +343,32 @@ struct GemmCfg {
   static constexpr bool kBmn = (KIND == kEpiStoreBf16 || KIND == kEpiRmwF32);
   static constexpr int kCtaN = PAIR ? BN / 2 : BN;     // B rows (N) held by this CTA
   static constexpr int kMmaM = PAIR ? 256 : 128;       // rows of one tile across the pair
+  // An MN-major B is staged as whole 64-column swizzle atoms; when kCtaN is not a
+  // multiple of 64 the MMA reads only the first kCtaN columns of the last atom
+  // (the rest is in-bounds neighbour data or TMA zero fill).
+  static constexpr int kBAtoms = (kCtaN + 63) / 64;
   static constexpr int kABytes = kBM * kBK * 2;
-  static constexpr int kBBytes = kCtaN * kBK * 2;
+  static constexpr int kBBytes = kBmn ? kBAtoms * 64 * kBK * 2 : kCtaN * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;               // landing in this CTA
   static constexpr int kTxBytes = (PAIR ? 2 : 1) * kStageBytes;       // counted on the MMA's barrier
   static constexpr int kEpiBytes =
-      (KIND == kEpiGrad || KIND == kEpiRmwF32) ? 4 * 4096 : (KIND == kEpiTopK ? kTopKMax * kBM * 8 : 0);
+      (KIND == kEpiGrad || KIND == kEpiRmwF32) ? 4 * 4096 : (KIND == kEpiTopK ? kTopKMax * kBM * 6 : 0);
   static constexpr int kBarBytes = 256;
   static constexpr int kSmemLimit = 232448;
   static constexpr int kStagesFit = (kSmemLimit - 1024 - kEpiBytes - kBarBytes) / kStageBytes;
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
   static constexpr int kSmem = 1024 + kStages * kStageBytes + kEpiBytes + kBarBytes;
   static constexpr uint32_t kIdesc = idesc_bf16_f32(kMmaM, BN, kAmn, kBmn);
-  static constexpr uint32_t kTmemCols = (2 * BN <= 256) ? 256u : 512u;
+  // the two accumulators sit at TMEM columns 0 and kAccStride (a power of two >= BN)
+  static constexpr int kAccStride = BN <= 128 ? 128 : 256;
+  static constexpr uint32_t kTmemCols = (2 * kAccStride <= 256) ? 256u : 512u;
   static constexpr int kAccEmptyArrivals = PAIR ? 8 : 4;
-  static_assert(kCtaN % 64 == 0 || !kBmn, "MN-major B needs whole 64-column atoms per CTA");
-  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
+  // tcgen05.mma kind::f16 with both operands in shared memory: N a multiple of 16 in
+  // [16, 256] for cta_group::2 (M = 256) and cta_group::1 (M = 128); BN % 16 also keeps
+  // each CTA's B coordinate (rank * kCtaN) on the 16-byte TMA boundary
+  static_assert(BN % 16 == 0 && BN >= 64 && BN <= 256, "BN");
+  static_assert(BN % 32 == 0 || KIND == kEpiStoreBf16 || KIND == kEpiRmwF32,
+                "the loss epilogues read whole 32-column TMEM chunks of a tile");
   static_assert(kStages >= 2, "stages");
 };
 
@@ -486,7 +496,7 @@ __global__ void __launch_bounds__(192, 1)
               }
               if (C::kBmn) {
 #pragma unroll
-                for (int q = 0; q < C::kCtaN / 64; ++q)
+                for (int q = 0; q < C::kBAtoms; ++q)
                   tma_load_2d_pair(b + q * 8192, &tmB, bar0, bcol + q * 64, kb * kBK);
               } else {
                 tma_load_2d_pair(b, &tmB, bar0, kb * kBK, bcol);
@@ -501,7 +511,7 @@ __global__ void __launch_bounds__(192, 1)
               }
               if (C::kBmn) {
 #pragma unroll
-                for (int q = 0; q < C::kCtaN / 64; ++q)
+                for (int q = 0; q < C::kBAtoms; ++q)
                   tma_load_2d(b + q * 8192, &tmB, &full[stage], bcol + q * 64, kb * kBK);
               } else {
                 tma_load_2d(b, &tmB, &full[stage], kb * kBK, bcol);
@@ -530,7 +540,7 @@ __global__ void __launch_bounds__(192, 1)
         for (int t = t0; t < t1; ++t) {
           if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, ab)) goto mma_done;
           tc_fence_after();
-          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::kAccStride);
           for (int kb = 0; kb < sc.k_blocks; ++kb) {
             if (!mbar_wait(&full[stage], phase, ab)) goto mma_done;
             tc_fence_after();
@@ -600,14 +610,18 @@ __global__ void __launch_bounds__(192, 1)
       const int row = row0 + row_local;
       const bool rv = row < ep.M;
       // teacher top-K: this thread's row owns column row_local of two [kTopKMax][128]
-      // shared arrays holding a min-heap ordered by (value, then larger index first)
+      // shared arrays holding a min-heap ordered by (value, then larger index first).
+      // Indices are kept relative to the unit's first column: a unit spans at most
+      // kTopKUnitTiles tiles, so 16 bits hold them and kTopKEmpty marks an empty slot
+      // (it also ranks after every real index, as the absolute sentinel does).
       float* hv = reinterpret_cast<float*>(wbuf_all) + row_local;
-      int* hi = reinterpret_cast<int*>(wbuf_all + kTopKMax * kBM * 4) + row_local;
+      uint16_t* hi = reinterpret_cast<uint16_t*>(wbuf_all + kTopKMax * kBM * 4) + row_local;
+      const int ubase = t0 * BN;
       float hroot = -INFINITY;
       if (KIND == kEpiTopK) {
         for (int k = 0; k < ep.topk_K; ++k) {
           hv[k * kBM] = -INFINITY;
-          hi[k * kBM] = kSentinel;
+          hi[k * kBM] = kTopKEmpty;
         }
       }
       const int64_t grow = ep.row_offset + row;
@@ -639,11 +653,14 @@ __global__ void __launch_bounds__(192, 1)
       for (int t = t0; t < t1; ++t) {
         if (!mbar_wait(&acc_full[acc], acc_phase, ab)) goto epi_done;
         tc_fence_after();
-        const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(acc * BN);
+        const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(acc * C::kAccStride);
+        // columns of this tile: [t * BN, col_lim); a last 32-column chunk that runs past
+        // BN reads unused TMEM columns, which the stores below skip
+        const int col_lim = min(ep.Ncols, t * BN + BN);
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = 0; c < (BN + 31) / 32; ++c) {
           const int col = t * BN + c * 32;
-          if (col >= ep.Ncols) break;
+          if (col >= col_lim) break;
           float v[32];
           tmem_ld32(tbase + c * 32, v);
           tmem_wait_ld();
@@ -705,7 +722,7 @@ __global__ void __launch_bounds__(192, 1)
               uint16_t* dst = ep.dH + grow * ep.ldo + col;
 #pragma unroll
               for (int g8 = 0; g8 < 4; ++g8) {
-                if (col + g8 * 8 + 8 <= ep.Ncols) {
+                if (col + g8 * 8 + 8 <= col_lim) {
                   uint4 pk;
                   pk.x = pack_bf16x2(v[g8 * 8 + 0], v[g8 * 8 + 1]);
                   pk.y = pack_bf16x2(v[g8 * 8 + 2], v[g8 * 8 + 3]);
@@ -730,7 +747,7 @@ __global__ void __launch_bounds__(192, 1)
               if (val > hroot) {
                 // replace the root (the smallest kept entry) and sift down; within a
                 // unit columns arrive in increasing order, so ties keep the earlier index
-                const int vi = col + j;
+                const int vi = col + j - ubase;
                 int pos = 0;
                 while (true) {
                   const int l = 2 * pos + 1;
@@ -749,11 +766,11 @@ __global__ void __launch_bounds__(192, 1)
                   }
                   if (cv > val || (cv == val && ci < vi)) break;   // child ranks above the new entry
                   hv[pos * kBM] = cv;
-                  hi[pos * kBM] = ci;
+                  hi[pos * kBM] = static_cast<uint16_t>(ci);
                   pos = c;
                 }
                 hv[pos * kBM] = val;
-                hi[pos * kBM] = vi;
+                hi[pos * kBM] = static_cast<uint16_t>(vi);
                 hroot = hv[0];
               }
             }
@@ -769,7 +786,7 @@ __global__ void __launch_bounds__(192, 1)
                            __float_as_uint(v[q4 * 4 + 2]), __float_as_uint(v[q4 * 4 + 3]));
             __syncwarp();
             const int wrow0 = row0 + q * 32;
-            const bool cv = (col + lane) < ep.Ncols;
+            const bool cv = (col + lane) < col_lim;
             float r[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i)
@@ -803,8 +820,9 @@ __global__ void __launch_bounds__(192, 1)
         const int64_t slot = (static_cast<int64_t>(u) * C::kMmaM + static_cast<int>(rank) * kBM + row_local) *
                              ep.topk_K;
         for (int k = 0; k < ep.topk_K; ++k) {
+          const int rel = hi[k * kBM];
           ep.part_tv[slot + k] = hv[k * kBM];
-          ep.part_ti[slot + k] = hi[k * kBM];
+          ep.part_ti[slot + k] = rel == kTopKEmpty ? kSentinel : ubase + rel;
         }
       }
       if (KIND == kEpiLse && rv) {
@@ -871,15 +889,32 @@ cudaError_t launch_gemm(int kind, int BN, bool pair, const CUtensorMap& tmA, con
                         const CUtensorMap& tmOut, const Sched& sc, const EpiParams& ep, int grid,
                         cudaStream_t stream) {
   if (pair) {
-    if (BN != 256) return cudaErrorInvalidValue;
+    // the loss and top-K GEMMs always use 256-wide tiles; dHidden / dW any pair width
+#define KDKL_PAIR_WIDTHS(KIND_)                                                                   \
+  switch (BN) {                                                                                   \
+    case 256: return launch_one<KIND_, 256, true>(tmA, tmB, tmOut, sc, ep, grid, stream);        \
+    case 240: return launch_one<KIND_, 240, true>(tmA, tmB, tmOut, sc, ep, grid, stream);        \
+    case 224: return launch_one<KIND_, 224, true>(tmA, tmB, tmOut, sc, ep, grid, stream);        \
+    case 192: return launch_one<KIND_, 192, true>(tmA, tmB, tmOut, sc, ep, grid, stream);        \
+    case 160: return launch_one<KIND_, 160, true>(tmA, tmB, tmOut, sc, ep, grid, stream);        \
+    case 128: return launch_one<KIND_, 128, true>(tmA, tmB, tmOut, sc, ep, grid, stream);        \
+    default: return cudaErrorInvalidValue;                                                        \
+  }
     switch (kind) {
-      case kEpiLse: return launch_one<kEpiLse, 256, true>(tmA, tmB, tmOut, sc, ep, grid, stream);
-      case kEpiGrad: return launch_one<kEpiGrad, 256, true>(tmA, tmB, tmOut, sc, ep, grid, stream);
-      case kEpiStoreBf16: return launch_one<kEpiStoreBf16, 256, true>(tmA, tmB, tmOut, sc, ep, grid, stream);
-      case kEpiRmwF32: return launch_one<kEpiRmwF32, 256, true>(tmA, tmB, tmOut, sc, ep, grid, stream);
-      case kEpiTopK: return launch_one<kEpiTopK, 256, true>(tmA, tmB, tmOut, sc, ep, grid, stream);
+      case kEpiLse:
+        if (BN != 256) return cudaErrorInvalidValue;
+        return launch_one<kEpiLse, 256, true>(tmA, tmB, tmOut, sc, ep, grid, stream);
+      case kEpiGrad:
+        if (BN != 256) return cudaErrorInvalidValue;
+        return launch_one<kEpiGrad, 256, true>(tmA, tmB, tmOut, sc, ep, grid, stream);
+      case kEpiTopK:
+        if (BN != 256) return cudaErrorInvalidValue;
+        return launch_one<kEpiTopK, 256, true>(tmA, tmB, tmOut, sc, ep, grid, stream);
+      case kEpiStoreBf16: KDKL_PAIR_WIDTHS(kEpiStoreBf16)
+      case kEpiRmwF32: KDKL_PAIR_WIDTHS(kEpiRmwF32)
       default: return cudaErrorInvalidValue;
     }
+#undef KDKL_PAIR_WIDTHS
   }
   switch (kind) {
     case kEpiLse:
@@ -931,7 +966,7 @@ cudaError_t launch_wait_selftest(uint32_t* flags, uint64_t limit_ns, uint64_t* w
 // top-K merge: one warp per row sorts the row's split heaps (bitonic, in
 // shared memory) by (value descending, index ascending) and keeps the first K
 // ============================================================================
-constexpr int kMergeCand = 1024;   // splits * K never exceeds this (the planner caps splits)
+constexpr int kMergeCand = kTopKMergeCand;   // splits * K never exceeds this (the planner caps splits)
 constexpr int kTopKMergeWarps = 4;
 
 __device__ __forceinline__ bool ranks_before(float av, int ai, float bv, int bi) {

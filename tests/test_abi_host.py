@@ -97,3 +97,63 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(K, "LIB_PATH", str(tmp_path / "nope.so"))
     with pytest.raises(RuntimeError, match="not built"):
         K.lib()
+
+
+def _dh_waves(N, d, bn, chunk, groups=74, rows=256):
+    """Waves of the dHidden GEMM over all chunks: ceil(row tiles x column tiles / CTA pairs) per chunk."""
+    nt = -(-d // bn)
+    total = 0
+    for c0 in range(0, N, chunk):
+        nc = min(chunk, N - c0)
+        total += -(-(-(-nc // rows) * nt) // groups)
+    return total
+
+
+def test_backward_plan_on_a_148_sm_device(lib):
+    # 8B-class head: 32 row tiles x 16 column tiles = 512 tiles = 6.9 waves of 74 pairs per chunk
+    assert K.kdkl_backward_plan(32768, 4096, 128256, 100, sm_count=148) == (256, 8192)
+    # d = 2880: 12 column tiles of 256; 30 row tiles per chunk give 360 dHidden tiles = 4.9 waves of
+    # 74 pairs, where 32 row tiles give 384 tiles = 5.2, i.e. 6 waves (86 against 96 in all)
+    assert K.kdkl_backward_plan(131072, 2880, 201088, 100, sm_count=148) == (256, 7680)
+    assert _dh_waves(131072, 2880, 256, 7680) == 86 and _dh_waves(131072, 2880, 256, 8192) == 96
+    # N below the chunk capacity: one chunk of N rounded up to 128 rows
+    assert K.kdkl_backward_plan(300, 200, 1001, 7, sm_count=148)[1] == 384
+
+
+def test_backward_plan_arguments(lib):
+    # an explicit chunk is kept (rounded up to 128 rows, at most N rounded up)
+    assert K.kdkl_backward_plan(32768, 4096, 128256, 100, chunk_tokens=1000, sm_count=148)[1] == 1024
+    assert K.kdkl_backward_plan(300, 200, 1001, 7, chunk_tokens=5000, sm_count=148)[1] == 384
+    # a forced tile width is kept; the chunk is planned for it
+    for bn in (256, 240, 224, 192, 160, 128):
+        assert K.kdkl_backward_plan(65536, 2880, 201088, 100, options=K.kdkl_options(bwd_tile_n=bn),
+                                    sm_count=148)[0] == bn
+    tn, ch = ctypes.c_int32(), ctypes.c_int64()
+    assert lib.kdkl_backward_plan(100, 64, 100, 10, 0, None, 148, None, ctypes.byref(ch)) == 1
+    assert lib.kdkl_backward_plan(100, 60, 100, 10, 0, None, 148, ctypes.byref(tn), ctypes.byref(ch)) == 2
+    assert lib.kdkl_backward_plan(100, 64, 100, 10, -1, None, 148, ctypes.byref(tn), ctypes.byref(ch)) == 2
+    bad = K.kdkl_options(bwd_tile_n=200)
+    assert lib.kdkl_backward_plan(100, 64, 100, 10, 0, ctypes.byref(bad), 148, ctypes.byref(tn),
+                                  ctypes.byref(ch)) == 4
+
+
+@pytest.mark.parametrize("sms", [148, 132, 2])
+def test_backward_plan_is_valid_everywhere(lib, sms):
+    for N in (1, 127, 256, 1000, 8192, 8193, 50000, 262144):
+        for d in (8, 200, 480, 896, 2048, 2880, 3584, 4096, 8192):
+            for V in (128, 32768, 201088):
+                bn, ch = K.kdkl_backward_plan(N, d, V, min(100, V), sm_count=sms)
+                assert bn in (256, 240, 224, 192, 160, 128)
+                n_up = -(-N // 128) * 128
+                assert ch % 128 == 0 and 128 <= ch <= min(8192, n_up)
+                assert K.kdkl_workspace_bytes(N, d, V, min(100, V)) >= K.kdkl_workspace_bytes(N, d, V, min(100, V), ch)
+
+
+def test_teacher_topk_vocabulary_limit(lib):
+    # each vocabulary split of the producer spans at most 255 tiles of 256 columns (16-bit heap
+    # indices), with at most floor(1024 / K) splits
+    assert K.kdkl_teacher_topk_workspace_bytes(4096, 4096, 522240, 128) > 0
+    assert K.kdkl_teacher_topk_workspace_bytes(4096, 4096, 522241, 128) == 0
+    assert K.kdkl_teacher_topk_workspace_bytes(4096, 4096, 652800, 100) > 0
+    assert K.kdkl_teacher_topk_workspace_bytes(4096, 4096, 652801, 100) == 0
+    assert K.kdkl_teacher_topk_workspace_bytes(4096, 4096, 201088, 128) > 0

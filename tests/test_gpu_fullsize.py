@@ -5,14 +5,21 @@ seconds, so it checks what it can compute one row at a time:
 
 * lse and dHidden on a seeded sample of rows (each sampled row's full
   vocabulary logits and gradient row, by the plain definition);
-* the loss, from the oracle's per-row teacher terms over every row
-  (sum P log P and the gathered logit sum_k P_k z[idx_k], both exact per row)
-  combined with the lse the GPU returns for every row, whose own accuracy the
-  sampled check establishes;
 * for dW, properties that hold at any size: every dW column sums to zero
   (each G row sums to zero), and <dW, W> = <dH, H> (both equal
   sum_{n,v} G[n, v] z[n, v]).
-Only the sampled rows and a few scalars leave the GPU.
+
+A second reference evaluates the same plain definition in float64 on the
+device with library routines only (torch matmul and logsumexp, no code of
+this library): the lse of every row, and dW on a seeded sample of vocabulary
+rows, which needs every token's softmax and hence every row's lse.  The
+teacher side of that reference (P_T per cached entry, the effective mask) is
+the CPU oracle's.  With it:
+* lse is compared on every row;
+* the loss is the oracle's per-row teacher terms over every row (sum P log P
+  and the gathered logit sum_k P_k z[idx_k], both exact per row) combined
+  with the float64 lse;
+* dW rows are compared element by element on the sample.
 """
 import numpy as np
 import pytest
@@ -26,6 +33,7 @@ from tests import gpu_harness as H
 pytestmark = [pytest.mark.gpu]
 
 SAMPLE = 96
+VOCAB_SAMPLE = 1024
 
 
 def _gather_term(x, W64, rows_per=512):
@@ -49,6 +57,45 @@ def _gather_term(x, W64, rows_per=512):
     return a, neg, m_eff
 
 
+def _device_fp64_reference(hidden, W, P, idx, m_eff, n_valid, vs, row_chunk=2048):
+    """lse for every row and dW[vs] in float64 on the device, from the plain definition:
+    z = H W^T, lse = logsumexp(z), G[n, v] = m_n (softmax(z)[n, v] - sum_{k: idx_k = v} P_k) / N_valid,
+    dW[v] = sum_n G[n, v] H[n] (the upstream gradient is 1)."""
+    dev = hidden.device
+    N = hidden.shape[0]
+    V = W.shape[0]
+    S = len(vs)
+    W64 = W.double()
+    vs_t = torch.from_numpy(vs).to(dev)
+    lse = torch.empty(N, dtype=torch.float64, device=dev)
+    zc = torch.empty(N, S, dtype=torch.float64, device=dev)
+    for r0 in range(0, N, row_chunk):
+        r1 = min(N, r0 + row_chunk)
+        z = hidden[r0:r1].double() @ W64.t()
+        lse[r0:r1] = torch.logsumexp(z, dim=1)
+        zc[r0:r1] = z[:, vs_t]
+        del z
+    del W64
+    # the teacher target restricted to the sampled columns
+    col = torch.full((V,), -1, dtype=torch.int64, device=dev)
+    col[vs_t] = torch.arange(S, device=dev)
+    idx_c = torch.from_numpy(np.clip(idx.astype(np.int64), 0, V - 1)).to(dev)
+    Pd = torch.from_numpy(P).to(dev)
+    j = col[idx_c]
+    hit = j >= 0
+    rows = torch.arange(N, device=dev)[:, None].expand_as(j)
+    target = torch.zeros(N * S, dtype=torch.float64, device=dev)
+    target.index_add_(0, (rows * S + j)[hit], Pd[hit])
+    m = torch.from_numpy(m_eff.astype(np.float64)).to(dev)
+    G = (torch.exp(zc - lse[:, None]) - target.view(N, S)) * (m / max(n_valid, 1))[:, None]
+    del zc, target
+    dW_s = torch.zeros(S, hidden.shape[1], dtype=torch.float64, device=dev)
+    for r0 in range(0, N, 8 * row_chunk):
+        r1 = min(N, r0 + 8 * row_chunk)
+        dW_s += G[r0:r1].t() @ hidden[r0:r1].double()
+    return lse.cpu().numpy(), dW_s.cpu().numpy()
+
+
 @pytest.mark.parametrize("name,N", [("8b", None), ("large_vocab", None), ("sweep", 16384), ("sweep", 262144)])
 def test_fullsize_sampled(name, N):
     w = synth.CONFIGS[name]
@@ -67,8 +114,10 @@ def test_fullsize_sampled(name, N):
     assert K.kdkl_read_device_flags(ws) == 0
     rows = synth.sample_rows(Nn, SAMPLE, seed=77)
     rows_t = torch.from_numpy(rows).cuda()
+    vs = np.unique(np.concatenate([synth.sample_rows(V, VOCAB_SAMPLE, seed=78), [0, V - 1]])).astype(np.int64)
     g_lse = lse.double().cpu().numpy()
     g_dH_rows = dH[rows_t].double().cpu().numpy()
+    g_dW_rows = dW[torch.from_numpy(vs).cuda()].double().cpu().numpy()
     # dW properties on the device, in float64
     dW64 = dW.double()
     col = dW64.sum(0)
@@ -85,9 +134,18 @@ def test_fullsize_sampled(name, N):
                   W_f64=W64)
     H.assert_lse(g_lse[rows], r.lse)
     H.assert_grad(g_dH_rows, r.dH, "dHidden (sampled rows)")
-    # loss: oracle per-row teacher terms over all rows + the GPU's lse
+    # float64 reference on the device: every row's lse, sampled dW rows
+    t = O.teacher_distribution(x.topk_idx, x.topk_logit, V, x.tau)
+    P = np.where(t.keep, t.P, 0.0)
+    m_eff = O.effective_mask(x.mask, t)
+    ref_lse, ref_dW_rows = _device_fp64_reference(dx.hidden, dx.W, P, x.topk_idx, m_eff, int(m_eff.sum()), vs)
+    torch.cuda.empty_cache()
+    np.testing.assert_allclose(ref_lse[rows], r.lse, rtol=0, atol=1e-9)   # the two references agree
+    H.assert_lse(g_lse, ref_lse)
+    H.assert_grad(g_dW_rows, ref_dW_rows, "dW (sampled vocabulary rows)")
+    # loss: oracle per-row teacher terms over all rows + the float64 lse
     a, neg, m_eff = _gather_term(x, W64)
-    ref_loss = float(((neg - a + g_lse) * m_eff).sum() / m_eff.sum())
+    ref_loss = float(((neg - a + ref_lse) * m_eff).sum() / m_eff.sum())
     H.assert_loss(float(loss.item()), ref_loss)
     # dW properties
     assert col_max <= 1e-3 * dW_max * np.sqrt(V)

@@ -108,3 +108,16 @@ def test_topk_fullsize_sampled():
     rows = synth.sample_rows(8192, 48, seed=530)
     exact = _check_rows(x, gi[rows], gv[rows], rows, 100)
     assert exact >= 24
+
+
+def test_topk_long_vocabulary_splits():
+    """38 row blocks of 256 at d = 64 over V = 60000 (235 column tiles): the planner keeps a
+    single vocabulary split (38 units already fill a wave as well as 76 would), so each row's
+    heap indices, kept relative to the split's first column, run past 32767."""
+    N = 38 * 256
+    x = synth.custom_inputs(N, 64, 60000, 1, seed=540, w_std=0.3)
+    gi, gv = _gpu_topk(x, 100)
+    assert gi.max() > 50000
+    rows = synth.sample_rows(N, 64, seed=541)
+    exact = _check_rows(x, gi[rows], gv[rows], rows, 100)
+    assert exact >= 48
