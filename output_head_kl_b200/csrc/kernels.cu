@@ -967,54 +967,140 @@ cudaError_t launch_wait_selftest(uint32_t* flags, uint64_t limit_ns, uint64_t* w
 // shared memory) by (value descending, index ascending) and keeps the first K
 // ============================================================================
 constexpr int kMergeCand = kTopKMergeCand;   // splits * K never exceeds this (the planner caps splits)
-constexpr int kTopKMergeWarps = 4;
+constexpr int kTopKMergeWarps = 8;
 
-__device__ __forceinline__ bool ranks_before(float av, int ai, float bv, int bi) {
-  return av > bv || (av == bv && ai < bi);
+// Orderable 64-bit key of a (logit, index) candidate: a larger key ranks
+// earlier (larger logit, then smaller index).  -0 is folded into +0 so that
+// equal logits tie on the index alone, as the comparison of values does.
+__device__ __forceinline__ uint64_t topk_key(float v, int idx) {
+  if (v == 0.0f) v = 0.0f;
+  uint32_t u = __float_as_uint(v);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return (static_cast<uint64_t>(u) << 32) | static_cast<uint64_t>(0xFFFFFFFFu - static_cast<uint32_t>(idx));
 }
 
+__device__ __forceinline__ float topk_key_value(uint64_t key) {
+  uint32_t u = static_cast<uint32_t>(key >> 32);
+  u = (u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u;
+  return __uint_as_float(u);
+}
+
+__device__ __forceinline__ int topk_key_index(uint64_t key) {
+  return static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(key));
+}
+
+// One warp per row: the row's S split heaps (S * K <= kMergeCand candidates,
+// K <= kTopKMax) are reduced to the K best, best first.  The K-th largest key
+// is found exactly by a radix select (one byte per pass, from the top, with a
+// 256-bin warp histogram); the keys above it, plus as many copies of it as are
+// still needed, are compacted with ballots and only those K are sorted.  The
+// K best of V >= K columns are always real entries, so empty heap slots
+// (-inf, sentinel index) never reach the output.
 __global__ void __launch_bounds__(kTopKMergeWarps * 32)
     topk_merge_kernel(const float* __restrict__ part_tv, const int* __restrict__ part_ti, int splits,
                       int rows_per_block, int K, int64_t N, int32_t* __restrict__ topk_idx,
                       float* __restrict__ topk_logit) {
-  __shared__ float s_v[kTopKMergeWarps][kMergeCand];
-  __shared__ int s_i[kTopKMergeWarps][kMergeCand];
+  constexpr int kPerLane = kMergeCand / 32;
+  __shared__ uint32_t s_hist[kTopKMergeWarps][256];
+  __shared__ uint64_t s_sel[kTopKMergeWarps][kTopKMax];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* sv = s_v[w];
-  int* si = s_i[w];
+  uint32_t* hist = s_hist[w];
+  uint64_t* sel = s_sel[w];
   const int C = splits * K;
-  int P = 32;
-  while (P < C) P <<= 1;
+  int P = 1;   // sort width of the K selected keys (a power of two <= kTopKMax)
+  while (P < K) P <<= 1;
   for (int64_t n = static_cast<int64_t>(blockIdx.x) * kTopKMergeWarps + w; n < N;
        n += static_cast<int64_t>(gridDim.x) * kTopKMergeWarps) {
     const int64_t rb = n / rows_per_block;
     const int r = static_cast<int>(n - rb * rows_per_block);
-    for (int c = lane; c < P; c += 32) {
+    // candidate c = j * K + k (split j, heap slot k) sits in lane c % 32 as key[c / 32];
+    // 0 ranks below every real key
+    uint64_t key[kPerLane];
+#pragma unroll
+    for (int i = 0; i < kPerLane; ++i) {
+      const int c = lane + 32 * i;
+      key[i] = 0;
       if (c < C) {
         const int j = c / K, k = c - j * K;
         const int64_t slot = ((rb * splits + j) * rows_per_block + r) * K + k;
-        sv[c] = part_tv[slot];
-        si[c] = part_ti[slot];
-      } else {
-        sv[c] = -INFINITY;
-        si[c] = kSentinel;
+        key[i] = topk_key(part_tv[slot], part_ti[slot]);
       }
     }
+    // radix select: after pass p, `prefix` holds the top p+1 bytes of the K-th
+    // largest key and `need` counts the keys still to take among those sharing them
+    uint64_t prefix = 0, pmask = 0;
+    int need = K;
+    for (int pass = 0; pass < 8; ++pass) {
+      const int shift = 56 - 8 * pass;
+      for (int b = lane; b < 256; b += 32) hist[b] = 0;
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < kPerLane; ++i)
+        if ((key[i] & pmask) == prefix) atomicAdd(&hist[(key[i] >> shift) & 0xFFu], 1u);
+      __syncwarp();
+      // lane l holds digits 255 - 8 l down to 248 - 8 l; lanes scan from the top
+      uint32_t cnt[8];
+      uint32_t tot = 0;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        cnt[t] = hist[255 - 8 * lane - t];
+        tot += cnt[t];
+      }
+      uint32_t incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const uint32_t excl = incl - tot;
+      const bool here = excl < static_cast<uint32_t>(need) && incl >= static_cast<uint32_t>(need);
+      const int src = __ffs(__ballot_sync(0xffffffffu, here)) - 1;
+      uint32_t digit = 0, above = excl;
+      if (here) {
+        bool found = false;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          if (!found) {
+            if (above + cnt[t] >= static_cast<uint32_t>(need)) {
+              digit = static_cast<uint32_t>(255 - 8 * lane - t);
+              found = true;
+            } else {
+              above += cnt[t];
+            }
+          }
+        }
+      }
+      digit = __shfl_sync(0xffffffffu, digit, src);
+      above = __shfl_sync(0xffffffffu, above, src);
+      need -= static_cast<int>(above);
+      prefix |= static_cast<uint64_t>(digit) << shift;
+      pmask |= 0xFFull << shift;
+      __syncwarp();
+    }
+    // keep the keys above the K-th, then `need` copies of it
+    const uint64_t kth = prefix;
+    int base = 0;
+#pragma unroll
+    for (int i = 0; i < kPerLane; ++i) {
+      const bool take = key[i] > kth;
+      const uint32_t b = __ballot_sync(0xffffffffu, take);
+      if (take) sel[base + __popc(b & ((1u << lane) - 1u))] = key[i];
+      base += __popc(b);
+    }
+    for (int k = base + lane; k < K; k += 32) sel[k] = kth;
+    for (int k = K + lane; k < P; k += 32) sel[k] = 0;
     __syncwarp();
+    // bitonic sort of the P selected keys, largest first
     for (int k2 = 2; k2 <= P; k2 <<= 1) {
       for (int j2 = k2 >> 1; j2 > 0; j2 >>= 1) {
         for (int i = lane; i < P; i += 32) {
           const int l = i ^ j2;
           if (l > i) {
-            const float a = sv[i], b = sv[l];
-            const int ai = si[i], bi = si[l];
-            const bool up = (i & k2) == 0;
-            const bool sw = up ? ranks_before(b, bi, a, ai) : ranks_before(a, ai, b, bi);
-            if (sw) {
-              sv[i] = b;
-              si[i] = bi;
-              sv[l] = a;
-              si[l] = ai;
+            const uint64_t a = sel[i], b = sel[l];
+            const bool first_block = (i & k2) == 0;
+            if (first_block ? (a < b) : (a > b)) {
+              sel[i] = b;
+              sel[l] = a;
             }
           }
         }
@@ -1022,8 +1108,9 @@ __global__ void __launch_bounds__(kTopKMergeWarps * 32)
       }
     }
     for (int k = lane; k < K; k += 32) {
-      topk_logit[n * K + k] = sv[k];
-      topk_idx[n * K + k] = si[k];
+      const uint64_t kk = sel[k];
+      topk_logit[n * K + k] = topk_key_value(kk);
+      topk_idx[n * K + k] = topk_key_index(kk);
     }
     __syncwarp();
   }

@@ -158,3 +158,26 @@ def test_ragged_cache_K255_with_duplicates():
     x.topk_idx[5, 200] = x.topk_idx[5, 3]
     g, r = _full_parity(x)
     assert g.flags == O.FLAG_IDX_DUP
+
+
+@pytest.mark.parametrize("N,d,V,Kc", [(130, 8, 100, 10), (3, 24, 257, 3), (5, 8, 40, 40)])
+def test_minimal_shapes(N, d, V, Kc):
+    """d = 8 (one 16-byte row: every box runs past d into zero fill), vocabularies narrower
+    than one 256-wide tile or one column past it, and a batch smaller than one row block."""
+    x = synth.custom_inputs(N, d, V, Kc, seed=150 + N, w_std=0.5, mask_frac=0.2 if N > 10 else 0.0)
+    _full_parity(x)
+
+
+def test_single_entry_vocabulary():
+    """V = K = 1: teacher and student both put all mass on the one entry, so the loss and
+    every gradient are zero up to rounding, and lse equals the one logit."""
+    x = synth.custom_inputs(70, 16, 1, 1, seed=160, w_std=0.5)
+    g = H.run_gpu(H.to_device(x))
+    r = _oracle(x)
+    assert r.loss == 0.0 and np.abs(r.dH).max() == 0.0
+    assert abs(g.loss) < 1e-6
+    H.assert_lse(g.lse, r.lse)
+    z = O.bf16_bits_to_f64(x.hidden_bits) @ O.bf16_bits_to_f64(x.W_bits)[0]
+    np.testing.assert_allclose(r.lse, z, rtol=0, atol=1e-12)
+    hw = np.abs(O.bf16_bits_to_f64(x.hidden_bits)).max() * np.abs(O.bf16_bits_to_f64(x.W_bits)).max()
+    assert np.abs(g.dH).max() <= 1e-5 * hw and np.abs(g.dW).max() <= 1e-5 * hw
