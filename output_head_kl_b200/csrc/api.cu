@@ -100,10 +100,13 @@ kdkl_status current_device(Device& dv) {
 // (single CTAs or CTA pairs), and keep at least enough splits that the hidden
 // rows in flight stay small next to L2.  `units_cap` bounds rb * splits.
 int pick_splits(int64_t rb, int vt, int ctas, int d, int64_t units_cap, int rows_per_block, int s_floor = 1) {
-  // Measured on the 8B-class head: the forward is fastest with about 9
-  // 256-row blocks (18 MB of hidden rows) in flight; 37 MB already thrashes L2.
+  // Fewer splits mean fewer passes over W, hence less DRAM traffic and power,
+  // but more hidden rows in flight.  Measured on B200 (forward, steady state):
+  // the fastest split counts were 2 at (N, d, V) = (131072, 2880, 201088),
+  // 3 at (131072, 4096, 128256) and 4 at (32768, 4096, 128256), i.e. 37-55 MB of
+  // hidden rows in flight, 3-9 % faster than at 18-20 MB.
   const double rows_bytes = static_cast<double>(rows_per_block) * d * 2.0;
-  const double budget = 20.0 * 1024 * 1024;
+  const double budget = 55.0 * 1024 * 1024;
   int s_min = static_cast<int>(std::ceil(ctas * rows_bytes / budget));
   if (s_min < s_floor) s_min = s_floor;
   if (s_min < 1) s_min = 1;
@@ -515,7 +518,7 @@ static kdkl_status forward_impl(const void* hidden, const void* W, const void* t
   sc.splits = splits;
   sc.n_tiles = vt;
   sc.k_blocks = (d + kBK - 1) / kBK;
-  sc.row_stream = 1;
+  sc.row_stream = kRowMajor;
   CUtensorMap tmA, tmB;
   if (!make_map(&tmA, hidden, d, N, d, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map(&tmB, W, d, V, d, kBK, pr.b_rows, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -617,7 +620,8 @@ static kdkl_status backward_impl(const void* hidden, const void* W, const void* 
     {
       const int64_t rbc = (nc + pg.rows - 1) / pg.rows;
       const int splits = pick_splits(rbc, vt, pg.groups, d, L.units_cap * kBM / pg.rows, pg.rows);
-      Sched sc{static_cast<int>(rbc * splits), splits, vt, (d + kBK - 1) / kBK, 1};
+      // a chunk's hidden rows fit in L2, so all its row blocks sweep each split together
+      Sched sc{static_cast<int>(rbc * splits), splits, vt, (d + kBK - 1) / kBK, kSplitMajor};
       EpiParams ep = ep0;
       ep.M = static_cast<int>(nc);
       ep.Ncols = V;
@@ -780,7 +784,7 @@ kdkl_status kdkl_teacher_topk(const void* hidden, const void* W, int64_t N, int3
   const int vt = (V + 255) / 256;
   const int splits = pick_splits(rb, vt, pr.groups, d, rb * L.s_cap, pr.rows,
                                  (vt + kTopKUnitTiles - 1) / kTopKUnitTiles);
-  Sched sc{static_cast<int>(rb * splits), splits, vt, (d + kBK - 1) / kBK, 1};
+  Sched sc{static_cast<int>(rb * splits), splits, vt, (d + kBK - 1) / kBK, kRowMajor};
   CUtensorMap tmA, tmB;
   if (!make_map(&tmA, hidden, d, N, d, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map(&tmB, W, d, V, d, kBK, pr.b_rows, CU_TENSOR_MAP_SWIZZLE_128B))

@@ -45,6 +45,15 @@ WsLayout make_layout(int64_t N, int32_t d, int32_t V, int32_t K, int64_t chunk_t
 //   row-stream mode: unit u -> row block u / splits, vocabulary tiles
 //     [(j * n_tiles) / splits, ((j + 1) * n_tiles) / splits) with j = u % splits.
 //   tile mode: unit u -> row block u / n_tiles, the single tile u % n_tiles.
+// Work units of a persistent GEMM launch, dealt round-robin to the CTA groups.
+//   row_stream = 0: one output tile per unit, u = row block * n_tiles + tile;
+//   row_stream = kRowMajor: a unit is (row block, vocabulary split) and sweeps the
+//     split's tiles, u = row block * splits + split (the row blocks in flight stay few);
+//   row_stream = kSplitMajor: the same units, u = split * row blocks + row block, so
+//     the groups running at once cover every row block of one split and share its
+//     W tiles (for launches whose row blocks all fit in L2).
+constexpr int kRowMajor = 1;
+constexpr int kSplitMajor = 2;
 struct Sched {
   int units;
   int splits;

@@ -374,8 +374,15 @@ struct GemmCfg {
 
 __device__ __forceinline__ void unit_range(const Sched& sc, int u, int& mb, int& t0, int& t1) {
   if (sc.row_stream) {
-    mb = u / sc.splits;
-    const int j = u - mb * sc.splits;
+    int j;
+    if (sc.row_stream == kSplitMajor) {
+      const int rb = sc.units / sc.splits;
+      j = u / rb;
+      mb = u - j * rb;
+    } else {
+      mb = u / sc.splits;
+      j = u - mb * sc.splits;
+    }
     t0 = static_cast<int>((static_cast<int64_t>(j) * sc.n_tiles) / sc.splits);
     t1 = static_cast<int>((static_cast<int64_t>(j + 1) * sc.n_tiles) / sc.splits);
   } else {
@@ -888,6 +895,9 @@ static cudaError_t launch_one(const CUtensorMap& tmA, const CUtensorMap& tmB, co
 cudaError_t launch_gemm(int kind, int BN, bool pair, const CUtensorMap& tmA, const CUtensorMap& tmB,
                         const CUtensorMap& tmOut, const Sched& sc, const EpiParams& ep, int grid,
                         cudaStream_t stream) {
+  // the forward and top-K epilogues index their per-unit partial results by unit
+  // number, which the merges read in row-major unit order
+  if ((kind == kEpiLse || kind == kEpiTopK) && sc.row_stream != kRowMajor) return cudaErrorInvalidValue;
   if (pair) {
     // the loss and top-K GEMMs always use 256-wide tiles; dHidden / dW any pair width
 #define KDKL_PAIR_WIDTHS(KIND_)                                                                   \
