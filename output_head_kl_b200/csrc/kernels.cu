@@ -973,8 +973,8 @@ cudaError_t launch_wait_selftest(uint32_t* flags, uint64_t limit_ns, uint64_t* w
 }
 
 // ============================================================================
-// top-K merge: one warp per row sorts the row's split heaps (bitonic, in
-// shared memory) by (value descending, index ascending) and keeps the first K
+// top-K merge: one warp per row keeps the K best of the row's split heaps,
+// ordered by value descending, then index ascending
 // ============================================================================
 constexpr int kMergeCand = kTopKMergeCand;   // splits * K never exceeds this (the planner caps splits)
 constexpr int kTopKMergeWarps = 8;
