@@ -44,15 +44,29 @@ def measured_peaks():
 
 
 # ----------------------------------------------------------------------------- ncu traffic record
-def kernel_sources_digest() -> str:
-    """sha256 over the CUDA sources; a traffic record only applies to the kernels it was taken on."""
+def _code_only(text: str) -> str:
+    """Source text without comments and with whitespace collapsed (what the compiler sees)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
+def kernel_sources_digest(read=None) -> str:
+    """sha256 over the code of the CUDA sources (comments and layout excluded); a traffic
+    record only applies to the kernels it was taken on.  `read(name)` overrides how a
+    source file's text is obtained (default: the working tree)."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "output_head_kl_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
         if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+            if read is None:
+                with open(os.path.join(csrc, name), encoding="utf-8") as f:
+                    text = f.read()
+            else:
+                text = read(name)
+            h.update(name.encode() + b"\0" + _code_only(text).encode())
     return h.hexdigest()
 
 
