@@ -340,7 +340,10 @@ def main_gpu(args, w: synth.Workload, N: int):
     idx = h_idx.to(dev)
     logit = h_logit.to(dev)
     mask = h_mask.to(dev)
-    ws_bytes = K.kdkl_workspace_bytes(Nn, d, V, Kc, args.chunk_tokens)
+    if args.fused_step and world > 1:
+        raise SystemExit("--fused-step is timed on one GPU")
+    ws_bytes = (K.kdkl_forward_backward_workspace_bytes(Nn, d, V, Kc, args.chunk_tokens) if args.fused_step
+                else K.kdkl_workspace_bytes(Nn, d, V, Kc, args.chunk_tokens))
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     loss = torch.empty(1, dtype=torch.float32, device=dev)
     lse = torch.empty(Nn, dtype=torch.float32, device=dev)
@@ -356,6 +359,10 @@ def main_gpu(args, w: synth.Workload, N: int):
 
     def step(bufs=None):
         hidden_, idx_, logit_, mask_ = bufs if bufs is not None else (hidden, idx, logit, mask)
+        if args.fused_step:
+            K.kdkl_forward_backward(hidden_, W, idx_, logit_, mask_, x.tau, loss, lse, dH, dW, ws,
+                                    chunk_tokens=args.chunk_tokens, stream=stream)
+            return
         K.kdkl_forward(hidden_, W, idx_, logit_, mask_, x.tau, loss, lse, ws, stream=stream)
         if world > 1:
             n_total.copy_(ws[4:8].view(torch.int32))
@@ -450,7 +457,7 @@ def main_gpu(args, w: synth.Workload, N: int):
         flops = synth.flops_fwd_bwd(Nn, d, V)
         tflops = flops / (ms_max * 1e-3) / 1e12
         # dominant kernel by total time; its algorithmic flops are 2 N d V per step
-        gemm_kinds = ("fwd_lse_gemm", "bwd_grad_gemm", "bwd_dhidden_gemm", "bwd_dw_gemm")
+        gemm_kinds = ("fwd_lse_gemm", "bwd_grad_gemm", "bwd_dhidden_gemm", "bwd_dw_gemm", "fused_fwd_gemm")
         dom = max(kt, key=lambda k: kt[k][1])
         launches, total_ms = kt[dom]
         if dom in gemm_kinds and launches:
@@ -482,12 +489,17 @@ def main_gpu(args, w: synth.Workload, N: int):
             "config": {"workload": w.name, "N": Nn, "d": d, "V": V, "K": Kc, "tau": x.tau,
                        "chunk_tokens": bwd_plan[1], "bwd_tile_n": bwd_plan[0],
                        "l2": "inputs larger than L2 (W alone is %.2f GB); no flush" % (V * d * 2 / 1e9),
-                       "parallelism": f"dp{world}" if world > 1 else "single"},
+                       "parallelism": f"dp{world}" if world > 1 else "single",
+                       "schedule": ("fused step: each chunk's logits computed once and kept for its gradient "
+                                    "(6 N d V flops executed)") if args.fused_step else
+                                   "kdkl_forward + kdkl_backward (the backward recomputes each chunk's logits)"},
             "tflops": tflops,
             "frac_of_bf16_peak": tflops / peaks["bf16_tflops"],
             "frac_of_bf16_peak_sustained": tflops / peaks["bf16_tflops_sustained"],
+            "executed_tflops": (0.75 if args.fused_step else 1.0) * tflops,
             "same_gpu_cublas": ref_gemm,
-            "frac_of_same_gpu_cublas": (tflops / ref_gemm["tflops"]) if ref_gemm else None,
+            "frac_of_same_gpu_cublas": ((0.75 if args.fused_step else 1.0) * tflops / ref_gemm["tflops"])
+                                       if ref_gemm else None,
             "peak_gb": peak_bytes / 1e9,
             "workspace_gb": ws_bytes / 1e9,
             "roofline": roof,
@@ -573,6 +585,8 @@ def main():
     ap.add_argument("--no-gemm-reference", action="store_true",
                     help="skip the same-GPU cuBLAS GEMM timed after the run (context only)")
     ap.add_argument("--topk", action="store_true", help="time the teacher top-K cache producer instead")
+    ap.add_argument("--fused-step", action="store_true",
+                    help="time kdkl_forward_backward (no logit recompute) instead of kdkl_forward + kdkl_backward")
     ap.add_argument("--record-traffic", metavar="NCU_CSV",
                     help="write profiles/traffic.json from an ncu dram__bytes capture of --config's workload")
     ap.add_argument("--sweep", action="store_true",

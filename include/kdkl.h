@@ -226,6 +226,36 @@ kdkl_status kdkl_backward_ex(const void* hidden, const void* W, const void* topk
                              size_t workspace_bytes, void* stream);
 
 /*
+ * Fused forward + backward, without the backward's logit recompute.  The pages'
+ * fused chunked loss recomputes each chunk's logits in the backward, so the
+ * projection runs twice and nothing N x V is ever stored (mind-verse.de
+ * article, section "Zwei systemische Optimierungen", the "Fused chunked KL"
+ * item).  This entry point computes each token chunk's logits once: one GEMM
+ * folds them into the online log-sum-exp and gather and also stores them (fp32)
+ * in a chunk buffer; once the chunk's rows have their lse, G is formed from the
+ * stored logits, and the chunk's dHidden and dW GEMMs run.  The chunk buffer is
+ * N-independent, so peak memory still grows only linearly with N, and the step
+ * does 6 N d V flops instead of 8 N d V.
+ * It computes what kdkl_forward_ex followed by kdkl_backward_ex compute with the
+ * same options: loss, lse, dHidden and dW (grad_loss, a device scalar or NULL = 1,
+ * must be known at call time).  Results agree with the separate calls up to
+ * rounding order: each row's log-sum-exp is merged from a different number of
+ * vocabulary splits.
+ *   workspace >= kdkl_forward_backward_workspace_bytes(N, d, V, K, chunk_tokens):
+ *     the loss workspace plus chunk x V fp32 logits (4.2 GB at 8192 x 128,256)
+ *   chunk_tokens is rounded up to a multiple of 256; 0 = the backward planner's
+ *     choice within the default capacity (kdkl_backward_plan reports it)
+ *   argument checks and errors as kdkl_forward_ex and kdkl_backward_ex; loss must
+ *     be non-NULL and 4-byte aligned
+ */
+size_t kdkl_forward_backward_workspace_bytes(int64_t N, int32_t d, int32_t V, int32_t K, int64_t chunk_tokens);
+kdkl_status kdkl_forward_backward(const void* hidden, const void* W, const void* topk_idx, const void* topk_logit,
+                                  const uint8_t* mask, int64_t N, int32_t d, int32_t V, int32_t K, float tau,
+                                  const kdkl_options* options, const float* grad_loss, float* loss, float* lse,
+                                  void* dHidden, float* dW, int64_t chunk_tokens, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/*
  * Teacher top-K cache producer: the step that builds the cache the loss reads.
  * The teacher runs once and, for each token position, only its K most likely
  * vocabulary entries are kept as (index, logit) pairs (mind-verse.de article,

@@ -95,6 +95,11 @@ def lib() -> ctypes.CDLL:
     L.kdkl_backward_ex.argtypes = [vp, vp, vp, vp, vp, i64, i32, i32, i32, f32, ctypes.POINTER(Options), vp, vp, vp,
                                    vp, i64, vp, sz, vp]
     L.kdkl_backward_ex.restype = ctypes.c_int
+    L.kdkl_forward_backward_workspace_bytes.argtypes = [i64, i32, i32, i32, i64]
+    L.kdkl_forward_backward_workspace_bytes.restype = sz
+    L.kdkl_forward_backward.argtypes = [vp, vp, vp, vp, vp, i64, i32, i32, i32, f32, ctypes.POINTER(Options), vp, vp,
+                                        vp, vp, vp, i64, vp, sz, vp]
+    L.kdkl_forward_backward.restype = ctypes.c_int
     L.kdkl_teacher_topk_workspace_bytes.argtypes = [i64, i32, i32, i32]
     L.kdkl_teacher_topk_workspace_bytes.restype = sz
     L.kdkl_teacher_topk.argtypes = [vp, vp, i64, i32, i32, i32, vp, vp, vp, sz, vp]
@@ -225,6 +230,29 @@ def kdkl_backward_ex(hidden, W, topk_idx, topk_logit, mask, tau, lse, grad_loss,
                                 _ptr(dW), int(chunk_tokens), _ptr(workspace), int(wsb), _stream(stream))
     if check:
         _check(st, "kdkl_backward_ex")
+    return st
+
+
+def kdkl_forward_backward_workspace_bytes(N: int, d: int, V: int, K: int, chunk_tokens: int = 0) -> int:
+    return int(lib().kdkl_forward_backward_workspace_bytes(N, d, V, K, chunk_tokens))
+
+
+def kdkl_forward_backward(hidden, W, topk_idx, topk_logit, mask, tau, loss, lse, dHidden, dW, workspace,
+                          options=None, *, grad_loss=None, chunk_tokens=0, N=None, d=None, V=None, K=None,
+                          workspace_bytes=None, stream=None, check=True) -> int:
+    """Calls kdkl_forward_backward: loss, lse, dHidden and dW in one call, each logit chunk computed once."""
+    N = hidden.shape[0] if N is None else N
+    d = hidden.shape[1] if d is None else d
+    V = W.shape[0] if V is None else V
+    K = topk_idx.shape[1] if K is None else K
+    wsb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    opt = ctypes.byref(options) if options is not None else None
+    st = lib().kdkl_forward_backward(_ptr(hidden), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask), int(N),
+                                     int(d), int(V), int(K), float(tau), opt, _ptr(grad_loss), _ptr(loss), _ptr(lse),
+                                     _ptr(dHidden), _ptr(dW), int(chunk_tokens), _ptr(workspace), int(wsb),
+                                     _stream(stream))
+    if check:
+        _check(st, "kdkl_forward_backward")
     return st
 
 

@@ -79,6 +79,20 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The same for an fp32 matrix.
+bool make_map_f32(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t pitch_elems,
+              uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {pitch_elems * 4};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // --------------------------------------------------------------- planner
 struct Device {
   int id = 0;
@@ -359,10 +373,12 @@ kdkl_status cuda_fail(cudaError_t e, const char* what) {
 }
 
 // ---------------------------------------------------------------- timing
-enum TimedKind { kTPrepass = 0, kTFwd, kTMerge, kTGrad, kTDh, kTDw, kTTopK, kTTopKMerge, kTKinds };
+enum TimedKind {
+  kTPrepass = 0, kTFwd, kTMerge, kTGrad, kTDh, kTDw, kTTopK, kTTopKMerge, kTFusedFwd, kTGPass, kTKinds
+};
 const char* const kTimedNames[kTKinds] = {"prepass",          "fwd_lse_gemm", "merge",         "bwd_grad_gemm",
                                           "bwd_dhidden_gemm", "bwd_dw_gemm",  "teacher_topk_gemm",
-                                          "teacher_topk_merge"};
+                                          "teacher_topk_merge", "fused_fwd_gemm", "fused_g_pass"};
 struct TimingRec {
   int kind;
   cudaEvent_t a, b;
@@ -541,7 +557,7 @@ static kdkl_status forward_impl(const void* hidden, const void* W, const void* t
          return launch_merge(ep.part_m, ep.part_s, ep.part_a, splits, pr.rows, c.opt.student_tau,
                              at<float>(workspace, L.negent), at<float>(workspace, L.wsum),
                              at<uint8_t>(workspace, L.rowmask), N, lse, loss, at<double>(workspace, L.blocksum),
-                             header, ep.n_valid, s);
+                             header, ep.n_valid, 0, 0, s);
        })) != cudaSuccess)
     return cuda_fail(e, "merge launch");
   return ok();
@@ -560,6 +576,49 @@ kdkl_status kdkl_forward_ex(const void* hidden, const void* W, const void* topk_
                             size_t workspace_bytes, void* stream) {
   return forward_impl(hidden, W, topk_idx, topk_logit, mask, N, d, V, K, tau, options, loss, lse, workspace,
                       workspace_bytes, stream);
+}
+
+// The chunk's dHidden rows (= G W, bf16) and its dW term (dW (+)= G^T hidden_chunk,
+// fp32 read-modify-write in chunk order; the first chunk overwrites), from the
+// chunk's G in the chunk buffer.
+static kdkl_status run_dh_dw(const EpiParams& ep0, const Pairing& pd, int bn, int32_t V, int32_t d, int64_t c0,
+                             int64_t nc, const CUtensorMap& tmG_k, const CUtensorMap& tmG_mn,
+                             const CUtensorMap& tmW_mn, const CUtensorMap& tmH_mn, void* dHidden, float* dW,
+                             cudaStream_t s) {
+  const int nt = (d + bn - 1) / bn;
+  cudaError_t e;
+  {
+    const int64_t rbc = (nc + pd.rows - 1) / pd.rows;
+    Sched sc{static_cast<int>(rbc * nt), 1, nt, static_cast<int>((V + kBK - 1) / kBK), 0};
+    EpiParams ep = ep0;
+    ep.M = static_cast<int>(nc);
+    ep.Ncols = d;
+    ep.row_offset = c0;
+    ep.dH = static_cast<uint16_t*>(dHidden);
+    ep.ldo = d;
+    const int grid = pd.grid(sc.units);
+    if ((e = timed(kTDh, s, [&] {
+           return launch_gemm(kEpiStoreBf16, bn, pd.pair, tmG_k, tmW_mn, tmG_k, sc, ep, grid, s);
+         })) != cudaSuccess)
+      return cuda_fail(e, "dHidden GEMM launch");
+  }
+  {
+    const int64_t vb = (V + pd.rows - 1) / pd.rows;
+    Sched sc{static_cast<int>(vb * nt), 1, nt, static_cast<int>((nc + kBK - 1) / kBK), 0};
+    EpiParams ep = ep0;
+    ep.M = V;
+    ep.Ncols = d;
+    ep.row_offset = 0;
+    ep.dW = dW;
+    ep.ldo = d;
+    ep.accumulate = c0 > 0 ? 1 : 0;
+    const int grid = pd.grid(sc.units);
+    if ((e = timed(kTDw, s, [&] {
+           return launch_gemm(kEpiRmwF32, bn, pd.pair, tmG_mn, tmH_mn, tmG_mn, sc, ep, grid, s);
+         })) != cudaSuccess)
+      return cuda_fail(e, "dW GEMM launch");
+  }
+  return KDKL_OK;
 }
 
 static kdkl_status backward_impl(const void* hidden, const void* W, const void* topk_idx, const void* topk_logit,
@@ -600,7 +659,6 @@ static kdkl_status backward_impl(const void* hidden, const void* W, const void* 
       !make_map(&tmW_mn, W, d, V, d, 64, kBK, CU_TENSOR_MAP_SWIZZLE_128B))
     return fail(KDKL_ERR_CUDA, "cuTensorMapEncodeTiled failed (W)");
   const int vt = (V + 255) / 256;
-  const int nt = (d + bn - 1) / bn;
   EpiParams ep0 = base_params(c, L);
   ep0.lse = lse;
   ep0.grad_loss = grad_loss;
@@ -632,39 +690,128 @@ static kdkl_status backward_impl(const void* hidden, const void* W, const void* 
            })) != cudaSuccess)
         return cuda_fail(e, "gradient GEMM launch");
     }
-    // (2) dHidden rows of the chunk = G W
+    // (2) dHidden rows of the chunk = G W; (3) dW (+)= G^T hidden_chunk
+    if ((st = run_dh_dw(ep0, pd, bn, V, d, c0, nc, tmG_k, tmG_mn, tmW_mn, tmH_mn, dHidden, dW, s)) != KDKL_OK)
+      return st;
+  }
+  return ok();
+}
+
+// ---------------------------------------------------------------- fused forward + backward
+// The step without the backward's logit recompute: per token chunk, one GEMM
+// computes the chunk's logits once, folds them into the online log-sum-exp and
+// gather (as the forward) and stores them (fp32) in a chunk buffer; the chunk's
+// merge completes its rows' lse (and the loss, after the last chunk); G is then
+// formed from the stored logits and the chunk's dHidden / dW GEMMs run as in the
+// backward.  The chunk buffer is N-independent, so peak memory stays linear in N.
+// Fused chunks are multiples of the merge's 256-row block.
+static int64_t fused_chunk_tokens(int64_t chunk_tokens) {
+  return chunk_tokens > 0 ? (chunk_tokens + 255) / 256 * 256 : 0;
+}
+
+static size_t fused_logit_offset(const WsLayout& L) { return align_up(L.total, 256); }
+
+static size_t fused_total(const WsLayout& L) {
+  return fused_logit_offset(L) + static_cast<size_t>(L.chunk) * L.Vp * sizeof(float);
+}
+
+static kdkl_status forward_backward_impl(const void* hidden, const void* W, const void* topk_idx,
+                                         const void* topk_logit, const uint8_t* mask, int64_t N, int32_t d,
+                                         int32_t V, int32_t K, float tau, const kdkl_options* options,
+                                         const float* grad_loss, float* loss, float* lse, void* dHidden, float* dW,
+                                         int64_t chunk_tokens, void* workspace, size_t workspace_bytes,
+                                         void* stream) {
+  const Common c{hidden,    W,         topk_idx,        topk_logit, mask, N, d, V, K, tau,
+                 workspace, workspace_bytes, options ? *options : default_options()};
+  const int64_t ct = fused_chunk_tokens(chunk_tokens);
+  WsLayout L;
+  kdkl_status st = check_common(c, ct, true, L);
+  if (st != KDKL_OK) return st;
+  if (workspace_bytes < fused_total(L))
+    return fail(KDKL_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, fused_total(L));
+  if (!loss || !lse || !dHidden || !dW) return fail(KDKL_ERR_NULL, "loss, lse, dHidden and dW must be non-NULL");
+  if (!aligned(loss, 4) || !aligned(lse, 4) || (grad_loss && !aligned(grad_loss, 4)))
+    return fail(KDKL_ERR_ALIGN, "loss, lse and grad_loss must be 4-byte aligned");
+  if (!aligned(dHidden, 16) || !aligned(dW, 16)) return fail(KDKL_ERR_ALIGN, "dHidden and dW must be 16-byte aligned");
+  Device dv;
+  if ((st = current_device(dv)) != KDKL_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (N == 0) {
+    if ((e = cudaMemsetAsync(workspace, 0, 256, s)) != cudaSuccess ||
+        (e = cudaMemsetAsync(loss, 0, sizeof(float), s)) != cudaSuccess ||
+        (e = cudaMemsetAsync(dW, 0, static_cast<size_t>(V) * d * sizeof(float), s)) != cudaSuccess)
+      return cuda_fail(e, "cudaMemsetAsync");
+    return ok();
+  }
+  if ((st = run_prepass(c, L, s)) != KDKL_OK) return st;
+
+  uint16_t* gbuf = at<uint16_t>(workspace, L.gbuf);
+  float* zbuf = at<float>(workspace, fused_logit_offset(L));
+  const Pairing pg = pairing(dv.sms, 256);
+  const BackwardPlan plan = plan_backward(N, d, V, L.chunk, ct == 0, c.opt.bwd_tile_n, dv.sms);
+  const int bn = plan.bn;
+  const int64_t chunk = plan.chunk;
+  const Pairing pd = pairing(dv.sms, bn);
+  CUtensorMap tmW_k, tmW_mn;
+  if (!make_map(&tmW_k, W, d, V, d, kBK, pg.b_rows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tmW_mn, W, d, V, d, 64, kBK, CU_TENSOR_MAP_SWIZZLE_128B))
+    return fail(KDKL_ERR_CUDA, "cuTensorMapEncodeTiled failed (W)");
+  const int vt = (V + 255) / 256;
+  EpiParams ep0 = base_params(c, L);
+  ep0.lse = lse;
+  ep0.grad_loss = grad_loss;
+  float* part = at<float>(workspace, L.partial);
+  const size_t plane = static_cast<size_t>(L.units_cap) * kBM;
+  uint32_t* header = at<uint32_t>(workspace, L.header);
+  const int64_t total_blocks = (N + 255) / 256;
+
+  for (int64_t c0 = 0; c0 < N; c0 += chunk) {
+    const int64_t nc = (N - c0) < chunk ? (N - c0) : chunk;
+    const void* hc = static_cast<const uint8_t*>(hidden) + static_cast<size_t>(c0) * d * 2;
+    CUtensorMap tmH_k, tmH_mn, tmZ, tmG_k, tmG_mn;
+    if (!make_map(&tmH_k, hc, d, nc, d, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tmH_mn, hc, d, nc, d, 64, kBK, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_f32(&tmZ, zbuf, V, nc, L.Vp, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tmG_k, gbuf, V, nc, L.Vp, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tmG_mn, gbuf, V, nc, L.Vp, 64, kBK, CU_TENSOR_MAP_SWIZZLE_128B))
+      return fail(KDKL_ERR_CUDA, "cuTensorMapEncodeTiled failed (chunk maps)");
+
+    // (1) the chunk's logits: online lse + gather partials, and the logits stored
+    const int64_t rbc = (nc + pg.rows - 1) / pg.rows;
+    const int splits = pick_splits(rbc, vt, pg.groups, d, L.units_cap * kBM / pg.rows, pg.rows);
     {
-      const int64_t rbc = (nc + pd.rows - 1) / pd.rows;
-      Sched sc{static_cast<int>(rbc * nt), 1, nt, static_cast<int>((V + kBK - 1) / kBK), 0};
+      Sched sc{static_cast<int>(rbc * splits), splits, vt, (d + kBK - 1) / kBK, kSplitMajor};
       EpiParams ep = ep0;
       ep.M = static_cast<int>(nc);
-      ep.Ncols = d;
+      ep.Ncols = V;
       ep.row_offset = c0;
-      ep.dH = static_cast<uint16_t*>(dHidden);
-      ep.ldo = d;
-      const int grid = pd.grid(sc.units);
-      if ((e = timed(kTDh, s, [&] {
-             return launch_gemm(kEpiStoreBf16, bn, pd.pair, tmG_k, tmW_mn, tmG_k, sc, ep, grid, s);
+      ep.part_m = part;
+      ep.part_s = part + plane;
+      ep.part_a = part + 2 * plane;
+      const int grid = pg.grid(sc.units);
+      if ((e = timed(kTFusedFwd, s, [&] {
+             return launch_gemm(kEpiLseStore, 256, pg.pair, tmH_k, tmW_k, tmZ, sc, ep, grid, s);
            })) != cudaSuccess)
-        return cuda_fail(e, "dHidden GEMM launch");
+        return cuda_fail(e, "fused forward GEMM launch");
     }
-    // (3) dW (+)= G^T hidden_chunk, in chunk order (first chunk overwrites)
-    {
-      const int64_t vb = (V + pd.rows - 1) / pd.rows;
-      Sched sc{static_cast<int>(vb * nt), 1, nt, static_cast<int>((nc + kBK - 1) / kBK), 0};
-      EpiParams ep = ep0;
-      ep.M = V;
-      ep.Ncols = d;
-      ep.row_offset = 0;
-      ep.dW = dW;
-      ep.ldo = d;
-      ep.accumulate = c0 > 0 ? 1 : 0;
-      const int grid = pd.grid(sc.units);
-      if ((e = timed(kTDw, s, [&] {
-             return launch_gemm(kEpiRmwF32, bn, pd.pair, tmG_mn, tmH_mn, tmG_mn, sc, ep, grid, s);
-           })) != cudaSuccess)
-        return cuda_fail(e, "dW GEMM launch");
-    }
+    // (2) the chunk's lse and loss terms (the last chunk's last block writes the loss)
+    if ((e = timed(kTMerge, s, [&] {
+           return launch_merge(part, part + plane, part + 2 * plane, splits, pg.rows, c.opt.student_tau,
+                               at<float>(workspace, L.negent) + c0, at<float>(workspace, L.wsum) + c0,
+                               at<uint8_t>(workspace, L.rowmask) + c0, nc, lse + c0, loss,
+                               at<double>(workspace, L.blocksum), header, ep0.n_valid, c0 / 256, total_blocks, s);
+         })) != cudaSuccess)
+      return cuda_fail(e, "merge launch");
+    // (3) G from the stored logits
+    if ((e = timed(kTGPass, s, [&] {
+           return launch_gpass(zbuf, L.Vp, gbuf, L.Vp, nc, V, c0, ep0.sidx, ep0.sprob, ep0.Kp, ep0.rowmask,
+                               ep0.wsum, lse, ep0.n_valid, grad_loss, c.opt.student_tau, s);
+         })) != cudaSuccess)
+      return cuda_fail(e, "G launch");
+    // (4) dHidden rows of the chunk = G W; (5) dW (+)= G^T hidden_chunk
+    if ((st = run_dh_dw(ep0, pd, bn, V, d, c0, nc, tmG_k, tmG_mn, tmW_mn, tmH_mn, dHidden, dW, s)) != KDKL_OK)
+      return st;
   }
   return ok();
 }
@@ -683,6 +830,20 @@ kdkl_status kdkl_backward_ex(const void* hidden, const void* W, const void* topk
                              float* dW, int64_t chunk_tokens, void* workspace, size_t workspace_bytes, void* stream) {
   return backward_impl(hidden, W, topk_idx, topk_logit, mask, N, d, V, K, tau, options, lse, grad_loss, dHidden, dW,
                        chunk_tokens, workspace, workspace_bytes, stream);
+}
+
+size_t kdkl_forward_backward_workspace_bytes(int64_t N, int32_t d, int32_t V, int32_t K, int64_t chunk_tokens) {
+  if (check_shapes(N, d, V, K, 1.0f) != KDKL_OK || chunk_tokens < 0) return 0;
+  return fused_total(make_layout(N, d, V, K, fused_chunk_tokens(chunk_tokens)));
+}
+
+kdkl_status kdkl_forward_backward(const void* hidden, const void* W, const void* topk_idx, const void* topk_logit,
+                                  const uint8_t* mask, int64_t N, int32_t d, int32_t V, int32_t K, float tau,
+                                  const kdkl_options* options, const float* grad_loss, float* loss, float* lse,
+                                  void* dHidden, float* dW, int64_t chunk_tokens, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  return forward_backward_impl(hidden, W, topk_idx, topk_logit, mask, N, d, V, K, tau, options, grad_loss, loss, lse,
+                               dHidden, dW, chunk_tokens, workspace, workspace_bytes, stream);
 }
 
 void kdkl_options_init(kdkl_options* options) {

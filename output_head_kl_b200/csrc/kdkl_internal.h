@@ -97,7 +97,9 @@ struct EpiParams {
   int* part_ti;
 };
 
-enum EpiKind { kEpiLse = 0, kEpiGrad = 1, kEpiStoreBf16 = 2, kEpiRmwF32 = 3, kEpiTopK = 4 };
+// kEpiLseStore: the forward's online log-sum-exp and gather (as kEpiLse), and
+// every fp32 logit tile also stored to a chunk buffer (fused forward + backward).
+enum EpiKind { kEpiLse = 0, kEpiGrad = 1, kEpiStoreBf16 = 2, kEpiRmwF32 = 3, kEpiTopK = 4, kEpiLseStore = 5 };
 
 // Teacher top-K producer: per-row min-heaps of up to kTopKMax entries live in
 // shared memory during the vocabulary sweep, with 16-bit indices relative to
@@ -117,10 +119,22 @@ cudaError_t launch_prepass(int cache_format, const void* topk_idx, const void* t
                            float beta, int* sidx, float* sprob, float* negent, float* wsum, uint8_t* rowmask,
                            int Kp, uint32_t* header, cudaStream_t stream);
 
+// G (bf16, row pitch ldg) from stored fp32 logits z (row pitch ldz) for the nc rows
+// of a chunk starting at global row row_offset; see gpass_kernel.
+cudaError_t launch_gpass(const float* z, int64_t ldz, uint16_t* G, int64_t ldg, int64_t nc, int V,
+                         int64_t row_offset, const int* sidx, const float* sprob, int Kp, const uint8_t* rowmask,
+                         const float* wsum, const float* lse, const uint32_t* n_valid, const float* grad_loss,
+                         float student_tau, cudaStream_t stream);
+
+// launch_merge: rows [0, N) of the pointers given (a chunk passes offset per-row
+// pointers); their 256-row block sums land at blocksum[block_base + b], and the
+// launch that completes block total_blocks - 1 of the step (0 = this launch's
+// grid) sums all total_blocks in order into *loss.
 cudaError_t launch_merge(const float* part_m, const float* part_s, const float* part_a, int splits,
                          int rows_per_block, float student_tau, const float* negent, const float* wsum,
                          const uint8_t* rowmask, int64_t N, float* lse, float* loss, double* blocksum,
-                         uint32_t* header, const uint32_t* n_valid, cudaStream_t stream);
+                         uint32_t* header, const uint32_t* n_valid, int64_t block_base, int64_t total_blocks,
+                         cudaStream_t stream);
 
 // GEMM kinds: A/B majorness and epilogue are fixed per kind.
 //   kEpiLse      : A = hidden K-major, B = W K-major, BN = 256, row-stream

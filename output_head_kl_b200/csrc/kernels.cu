@@ -266,7 +266,7 @@ __global__ void __launch_bounds__(kMergeThreads)
                  const float* __restrict__ negent, const float* __restrict__ wsum,
                  const uint8_t* __restrict__ rowmask, int64_t N, float* __restrict__ lse,
                  float* __restrict__ loss, double* __restrict__ blocksum, uint32_t* __restrict__ header,
-                 const uint32_t* __restrict__ n_valid) {
+                 const uint32_t* __restrict__ n_valid, int64_t block_base, int64_t total_blocks) {
   __shared__ double s_red[kMergeThreads / 32];
   __shared__ bool s_last;
   const int64_t n = static_cast<int64_t>(blockIdx.x) * kMergeThreads + threadIdx.x;
@@ -297,17 +297,17 @@ __global__ void __launch_bounds__(kMergeThreads)
   if (threadIdx.x == 0) {
     double t = 0.0;
     for (int i = 0; i < kMergeThreads / 32; ++i) t += s_red[i];
-    blocksum[blockIdx.x] = t;
+    blocksum[block_base + blockIdx.x] = t;
     __threadfence();
     const uint32_t ticket = atomicAdd(&header[2], 1u);
-    s_last = (ticket == gridDim.x - 1);
+    s_last = (static_cast<int64_t>(ticket) == total_blocks - 1);
   }
   __syncthreads();
   if (s_last && threadIdx.x == 0) {
     __threadfence();
     double t = 0.0;
     const volatile double* bs = blocksum;
-    for (unsigned i = 0; i < gridDim.x; ++i) t += bs[i];
+    for (int64_t i = 0; i < total_blocks; ++i) t += bs[i];
     const uint32_t nv = *reinterpret_cast<const volatile uint32_t*>(n_valid);
     loss[0] = nv > 0 ? static_cast<float>(t / static_cast<double>(nv)) : 0.f;
     header[2] = 0;
@@ -317,11 +317,13 @@ __global__ void __launch_bounds__(kMergeThreads)
 cudaError_t launch_merge(const float* part_m, const float* part_s, const float* part_a, int splits,
                          int rows_per_block, float student_tau, const float* negent, const float* wsum,
                          const uint8_t* rowmask, int64_t N, float* lse, float* loss, double* blocksum,
-                         uint32_t* header, const uint32_t* n_valid, cudaStream_t stream) {
+                         uint32_t* header, const uint32_t* n_valid, int64_t block_base, int64_t total_blocks,
+                         cudaStream_t stream) {
   const int grid = static_cast<int>((N + kMergeThreads - 1) / kMergeThreads);
+  if (total_blocks <= 0) total_blocks = grid;
   merge_kernel<<<grid, kMergeThreads, 0, stream>>>(part_m, part_s, part_a, splits, rows_per_block,
                                                    1.0f / student_tau, negent, wsum, rowmask, N, lse, loss,
-                                                   blocksum, header, n_valid);
+                                                   blocksum, header, n_valid, block_base, total_blocks);
   return cudaGetLastError();
 }
 
@@ -351,8 +353,12 @@ struct GemmCfg {
   static constexpr int kBBytes = kBmn ? kBAtoms * 64 * kBK * 2 : kCtaN * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;               // landing in this CTA
   static constexpr int kTxBytes = (PAIR ? 2 : 1) * kStageBytes;       // counted on the MMA's barrier
-  static constexpr int kEpiBytes =
-      (KIND == kEpiGrad || KIND == kEpiRmwF32) ? 4 * 4096 : (KIND == kEpiTopK ? kTopKMax * kBM * 6 : 0);
+  // per-epilogue-warp staging: grad 2 x 2 KB (32 x 32 bf16), dW 4 KB (32 x 32 fp32),
+  // stored logits 2 x 4 KB (32 x 32 fp32); top-K: the heaps of all 128 rows
+  static constexpr int kEpiWarpBytes = (KIND == kEpiLseStore) ? 8192 : 4096;
+  static constexpr int kEpiBytes = (KIND == kEpiGrad || KIND == kEpiRmwF32 || KIND == kEpiLseStore)
+                                       ? 4 * kEpiWarpBytes
+                                       : (KIND == kEpiTopK ? kTopKMax * kBM * 6 : 0);
   static constexpr int kBarBytes = 256;
   static constexpr int kSmemLimit = 232448;
   static constexpr int kStagesFit = (kSmemLimit - 1024 - kEpiBytes - kBarBytes) / kStageBytes;
@@ -372,9 +378,11 @@ struct GemmCfg {
   static_assert(kStages >= 2, "stages");
 };
 
-__device__ __forceinline__ void unit_range(const Sched& sc, int u, int& mb, int& t0, int& t1) {
+// Unit u -> row block mb, vocabulary split j (row-stream units; 0 otherwise) and
+// its tile range [t0, t1).
+__device__ __forceinline__ void unit_range(const Sched& sc, int u, int& mb, int& j, int& t0, int& t1) {
+  j = 0;
   if (sc.row_stream) {
-    int j;
     if (sc.row_stream == kSplitMajor) {
       const int rb = sc.units / sc.splits;
       j = u / rb;
@@ -423,6 +431,7 @@ __global__ void __launch_bounds__(192, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmOut, const Sched sc, const EpiParams ep) {
   using C = GemmCfg<KIND, BN, PAIR>;
+  constexpr bool kLseLike = (KIND == kEpiLse || KIND == kEpiLseStore);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -458,7 +467,7 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
-    if (KIND == kEpiGrad) tma_prefetch_desc(&tmOut);
+    if (KIND == kEpiGrad || KIND == kEpiLseStore) tma_prefetch_desc(&tmOut);
   }
   if (warp == 1) {
     if (PAIR) {
@@ -482,8 +491,8 @@ __global__ void __launch_bounds__(192, 1)
       int stage = 0;
       uint32_t phase = 0;
       for (int u = group; u < sc.units; u += ngroups) {
-        int mb, t0, t1;
-        unit_range(sc, u, mb, t0, t1);
+        int mb, uj, t0, t1;
+        unit_range(sc, u, mb, uj, t0, t1);
         const int arow = mb * C::kMmaM + static_cast<int>(rank) * kBM;   // this CTA's A rows
         for (int t = t0; t < t1; ++t) {
           const int bcol = t * BN + static_cast<int>(rank) * C::kCtaN;  // this CTA's B rows (N)
@@ -542,8 +551,8 @@ __global__ void __launch_bounds__(192, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       for (int u = group; u < sc.units; u += ngroups) {
-        int mb, t0, t1;
-        unit_range(sc, u, mb, t0, t1);
+        int mb, uj, t0, t1;
+        unit_range(sc, u, mb, uj, t0, t1);
         for (int t = t0; t < t1; ++t) {
           if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, ab)) goto mma_done;
           tc_fence_after();
@@ -607,12 +616,15 @@ __global__ void __launch_bounds__(192, 1)
       g_scale = nv > 0 ? g * ep.inv_tau_s / static_cast<float>(nv) : 0.f;
     }
     const float es = ep.exp_scale;   // log2(e) / tau_s
-    uint8_t* wbuf = sEpi + (warp - 2) * 4096;   // this warp's staging (grad: 2 x 2 KB, dW: 4 KB)
+    uint8_t* wbuf = sEpi + (warp - 2) * C::kEpiWarpBytes;   // this warp's staging
     uint8_t* wbuf_all = sEpi;                    // top-K heaps of all 128 rows
     int sbuf = 0;
     for (int u = group; u < sc.units; u += ngroups) {
-      int mb, t0, t1;
-      unit_range(sc, u, mb, t0, t1);
+      int mb, uj, t0, t1;
+      unit_range(sc, u, mb, uj, t0, t1);
+      // this unit's partial-result slot: (row block, split) in row-major order, whatever
+      // order the units are dealt in (the merges read them that way)
+      const int64_t uslot = static_cast<int64_t>(mb) * sc.splits + uj;
       const int row0 = mb * C::kMmaM + static_cast<int>(rank) * kBM;   // first row of this CTA
       const int row = row0 + row_local;
       const bool rv = row < ep.M;
@@ -639,7 +651,7 @@ __global__ void __launch_bounds__(192, 1)
       float nxtp = 0.f;
       const int* lst = nullptr;
       const float* lsp = nullptr;
-      if (KIND == kEpiLse || KIND == kEpiGrad) {
+      if (kLseLike || KIND == kEpiGrad) {
         bool live = rv;
         if (KIND == kEpiGrad) {
           cn = (rv && ep.rowmask[grow]) ? g_scale : 0.f;
@@ -671,7 +683,29 @@ __global__ void __launch_bounds__(192, 1)
           float v[32];
           tmem_ld32(tbase + c * 32, v);
           tmem_wait_ld();
-          if (KIND == kEpiLse) {
+          if (kLseLike) {
+            if (KIND == kEpiLseStore) {
+              // stage the warp's 32 rows x 32 fp32 logits (128-byte swizzle: 16-byte
+              // chunk q of row r at chunk q ^ (r & 7)) and store them with TMA; columns
+              // past V and rows past the chunk are clipped by the tensor map
+              uint8_t* buf = wbuf + sbuf * 4096;
+              if (lane == 0) bulk_wait_read<1>();
+              __syncwarp();
+              const uint32_t sw = static_cast<uint32_t>(lane & 7);
+              const uint32_t row_addr = smem_u32(buf) + static_cast<uint32_t>(lane) * 128u;
+#pragma unroll
+              for (int c16 = 0; c16 < 8; ++c16)
+                st_shared_v4(row_addr + ((static_cast<uint32_t>(c16) ^ sw) << 4), __float_as_uint(v[c16 * 4 + 0]),
+                             __float_as_uint(v[c16 * 4 + 1]), __float_as_uint(v[c16 * 4 + 2]),
+                             __float_as_uint(v[c16 * 4 + 3]));
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&tmOut, buf, col, row0 + q * 32);
+                bulk_commit();
+              }
+              sbuf ^= 1;
+            }
             if (col + 32 > ep.Ncols) {
 #pragma unroll
               for (int j = 0; j < 32; ++j)
@@ -824,7 +858,7 @@ __global__ void __launch_bounds__(192, 1)
         if (acc == 0) acc_phase ^= 1u;
       }
       if (KIND == kEpiTopK && rv) {
-        const int64_t slot = (static_cast<int64_t>(u) * C::kMmaM + static_cast<int>(rank) * kBM + row_local) *
+        const int64_t slot = (uslot * C::kMmaM + static_cast<int>(rank) * kBM + row_local) *
                              ep.topk_K;
         for (int k = 0; k < ep.topk_K; ++k) {
           const int rel = hi[k * kBM];
@@ -832,15 +866,15 @@ __global__ void __launch_bounds__(192, 1)
           ep.part_ti[slot + k] = rel == kTopKEmpty ? kSentinel : ubase + rel;
         }
       }
-      if (KIND == kEpiLse && rv) {
-        const int64_t slot = static_cast<int64_t>(u) * C::kMmaM + static_cast<int>(rank) * kBM + row_local;
+      if (kLseLike && rv) {
+        const int64_t slot = uslot * C::kMmaM + static_cast<int>(rank) * kBM + row_local;
         ep.part_m[slot] = m_run;
         ep.part_s[slot] = s_run;
         ep.part_a[slot] = a_run;
       }
     }
   epi_done:
-    if (KIND == kEpiGrad) {
+    if (KIND == kEpiGrad || KIND == kEpiLseStore) {
       if (lane == 0) bulk_wait<0>();
       __syncwarp();
     }
@@ -895,9 +929,6 @@ static cudaError_t launch_one(const CUtensorMap& tmA, const CUtensorMap& tmB, co
 cudaError_t launch_gemm(int kind, int BN, bool pair, const CUtensorMap& tmA, const CUtensorMap& tmB,
                         const CUtensorMap& tmOut, const Sched& sc, const EpiParams& ep, int grid,
                         cudaStream_t stream) {
-  // the forward and top-K epilogues index their per-unit partial results by unit
-  // number, which the merges read in row-major unit order
-  if ((kind == kEpiLse || kind == kEpiTopK) && sc.row_stream != kRowMajor) return cudaErrorInvalidValue;
   if (pair) {
     // the loss and top-K GEMMs always use 256-wide tiles; dHidden / dW any pair width
 #define KDKL_PAIR_WIDTHS(KIND_)                                                                   \
@@ -914,6 +945,9 @@ cudaError_t launch_gemm(int kind, int BN, bool pair, const CUtensorMap& tmA, con
       case kEpiLse:
         if (BN != 256) return cudaErrorInvalidValue;
         return launch_one<kEpiLse, 256, true>(tmA, tmB, tmOut, sc, ep, grid, stream);
+      case kEpiLseStore:
+        if (BN != 256) return cudaErrorInvalidValue;
+        return launch_one<kEpiLseStore, 256, true>(tmA, tmB, tmOut, sc, ep, grid, stream);
       case kEpiGrad:
         if (BN != 256) return cudaErrorInvalidValue;
         return launch_one<kEpiGrad, 256, true>(tmA, tmB, tmOut, sc, ep, grid, stream);
@@ -929,6 +963,8 @@ cudaError_t launch_gemm(int kind, int BN, bool pair, const CUtensorMap& tmA, con
   switch (kind) {
     case kEpiLse:
       return launch_one<kEpiLse, 256, false>(tmA, tmB, tmOut, sc, ep, grid, stream);
+    case kEpiLseStore:
+      return launch_one<kEpiLseStore, 256, false>(tmA, tmB, tmOut, sc, ep, grid, stream);
     case kEpiGrad:
       return launch_one<kEpiGrad, 256, false>(tmA, tmB, tmOut, sc, ep, grid, stream);
     case kEpiStoreBf16:
@@ -969,6 +1005,108 @@ __global__ void wait_selftest_kernel(uint32_t* flags, uint64_t limit_ns, uint64_
 
 cudaError_t launch_wait_selftest(uint32_t* flags, uint64_t limit_ns, uint64_t* waited_ns, cudaStream_t stream) {
   wait_selftest_kernel<<<1, 32, 0, stream>>>(flags, limit_ns, waited_ns);
+  return cudaGetLastError();
+}
+
+// ============================================================================
+// G from stored logits (fused forward + backward).  For each row n of a chunk:
+//   G[n, v] = c_n (w_n 2^{z[n, v] log2e / tau_s - lse_n log2e} - target[n, v])  (bf16),
+// c_n = m_n g / (tau_s N_valid), with the gradient epilogue's instructions in the
+// same order, so that for the same z and lse the result is the same bits.  One
+// block per row; warp w covers the 128-column groups w, w + 8, ... (lane l holds
+// 4 columns), and the row's sorted target list is walked forward once per warp.
+// ============================================================================
+constexpr int kGPassThreads = 256;
+
+__global__ void __launch_bounds__(kGPassThreads)
+    gpass_kernel(const float* __restrict__ z, int64_t ldz, uint16_t* __restrict__ G, int64_t ldg, int V,
+                 int64_t row_offset, const int* __restrict__ sidx, const float* __restrict__ sprob, int Kp,
+                 const uint8_t* __restrict__ rowmask, const float* __restrict__ wsum,
+                 const float* __restrict__ lse, const uint32_t* __restrict__ n_valid,
+                 const float* __restrict__ grad_loss, float inv_tau_s, float exp_scale) {
+  const int64_t n = blockIdx.x;
+  const int64_t grow = row_offset + n;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t nv = *n_valid;
+  const float g = grad_loss ? *grad_loss : 1.0f;
+  const float g_scale = nv > 0 ? g * inv_tau_s / static_cast<float>(nv) : 0.f;
+  const float cn = rowmask[grow] ? g_scale : 0.f;
+  uint16_t* grow_out = G + n * ldg;
+  const float* zrow = z + n * ldz;
+  const int groups = (V + 127) / 128;
+  if (cn == 0.f) {
+    for (int gi = warp; gi < groups; gi += kGPassThreads / 32) {
+      const int c0 = gi * 128 + lane * 4;
+      if (c0 + 3 < V) {
+        *reinterpret_cast<uint2*>(grow_out + c0) = make_uint2(0u, 0u);
+      } else {
+        for (int j = 0; j < 4; ++j)
+          if (c0 + j < V) grow_out[c0 + j] = 0;
+      }
+    }
+    return;
+  }
+  const float es = exp_scale;
+  const float lse_l2 = lse[grow] * kLog2e;
+  const float cnw = cn * wsum[grow];
+  const int* lst = sidx + grow * Kp;
+  const float* lsp = sprob + grow * Kp;
+  // four 128-column groups per pass: their loads are all in flight before any is used
+  constexpr int kStride = kGPassThreads / 32;
+  constexpr int kU = 4;
+  int kpos = lower_bound_list(lst, Kp, warp * 128);
+  for (int gb = warp; gb < groups; gb += kStride * kU) {
+    float v[kU][4];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int c0 = (gb + u * kStride) * 128 + lane * 4;
+      if (c0 + 3 < V) {
+        const float4 q = *reinterpret_cast<const float4*>(zrow + c0);
+        v[u][0] = q.x;
+        v[u][1] = q.y;
+        v[u][2] = q.z;
+        v[u][3] = q.w;
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[u][j] = (c0 + j < V) ? zrow[c0 + j] : 0.f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int gi = gb + u * kStride;
+      if (gi >= groups) break;
+      const int g0 = gi * 128;
+      const int c0 = g0 + lane * 4;
+      float gv[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) gv[j] = cnw * ex2_approx(fmaf(v[u][j], es, -lse_l2));
+      while (lst[kpos] < g0) ++kpos;
+      for (int k = kpos; lst[k] < g0 + 128; ++k) {
+        const uint32_t off = static_cast<uint32_t>(lst[k] - c0);
+        const float cp = cn * lsp[k];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) gv[j] = (off == static_cast<uint32_t>(j)) ? gv[j] - cp : gv[j];
+      }
+      if (c0 + 3 < V) {
+        *reinterpret_cast<uint2*>(grow_out + c0) =
+            make_uint2(pack_bf16x2(gv[0], gv[1]), pack_bf16x2(gv[2], gv[3]));
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (c0 + j < V) grow_out[c0 + j] = static_cast<uint16_t>(pack_bf16x2(gv[j], 0.f) & 0xFFFFu);
+      }
+    }
+  }
+}
+
+cudaError_t launch_gpass(const float* z, int64_t ldz, uint16_t* G, int64_t ldg, int64_t nc, int V,
+                         int64_t row_offset, const int* sidx, const float* sprob, int Kp, const uint8_t* rowmask,
+                         const float* wsum, const float* lse, const uint32_t* n_valid, const float* grad_loss,
+                         float student_tau, cudaStream_t stream) {
+  if (nc <= 0) return cudaSuccess;
+  gpass_kernel<<<static_cast<unsigned>(nc), kGPassThreads, 0, stream>>>(
+      z, ldz, G, ldg, V, row_offset, sidx, sprob, Kp, rowmask, wsum, lse, n_valid, grad_loss, 1.0f / student_tau,
+      1.4426950408889634f / student_tau);
   return cudaGetLastError();
 }
 
