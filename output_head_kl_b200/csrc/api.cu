@@ -723,7 +723,8 @@ static kdkl_status forward_backward_impl(const void* hidden, const void* W, cons
                                          void* stream) {
   const Common c{hidden,    W,         topk_idx,        topk_logit, mask, N, d, V, K, tau,
                  workspace, workspace_bytes, options ? *options : default_options()};
-  const int64_t ct = fused_chunk_tokens(chunk_tokens);
+  // a negative chunk_tokens reaches check_common unrounded and is refused there
+  const int64_t ct = chunk_tokens < 0 ? chunk_tokens : fused_chunk_tokens(chunk_tokens);
   WsLayout L;
   kdkl_status st = check_common(c, ct, true, L);
   if (st != KDKL_OK) return st;

@@ -157,3 +157,22 @@ def test_teacher_topk_vocabulary_limit(lib):
     assert K.kdkl_teacher_topk_workspace_bytes(4096, 4096, 652800, 100) > 0
     assert K.kdkl_teacher_topk_workspace_bytes(4096, 4096, 652801, 100) == 0
     assert K.kdkl_teacher_topk_workspace_bytes(4096, 4096, 201088, 128) > 0
+
+
+def test_forward_backward_argument_checks(lib):
+    N, d, V, Kc = 256, 256, 4096, 16
+    need = K.kdkl_forward_backward_workspace_bytes(N, d, V, Kc)
+    # the fused step's workspace is the loss workspace plus the chunk's fp32 logits
+    assert need >= K.kdkl_workspace_bytes(N, d, V, Kc) + 256 * V * 4
+    assert K.kdkl_forward_backward_workspace_bytes(N, 12, V, Kc) == 0          # d % 8
+
+    def fb(**kw):
+        a = dict(loss=0x60000, lse=0x70000, dH=0x90000, dW=0xA0000, chunk=0, ws_bytes=need)
+        a.update(kw)
+        return lib.kdkl_forward_backward(0x10000, 0x20000, 0x30000, 0x40000, 0x50000, N, d, V, Kc, 1.0, None, None,
+                                         a["loss"], a["lse"], a["dH"], a["dW"], a["chunk"], 0x80000, a["ws_bytes"],
+                                         None)
+    assert fb(loss=None) == 1
+    assert fb(dW=0xA0004) == 3
+    assert fb(chunk=-1) == 2
+    assert fb(ws_bytes=need - 1) == 5 and "workspace" in K.kdkl_last_error()
