@@ -249,6 +249,21 @@ def blas_threads() -> int:
     return os.cpu_count() or 1
 
 
+def host_cpu_info() -> dict:
+    """The BLAS library numpy calls and the CPU cores this process may run on."""
+    blas = None
+    try:
+        dep = np.show_config(mode="dicts").get("Build Dependencies", {}).get("blas", {})
+        blas = f"{dep.get('name', '?')} {dep.get('version', '')}".strip()
+    except Exception:
+        pass
+    try:
+        affinity = len(os.sched_getaffinity(0))
+    except AttributeError:
+        affinity = os.cpu_count()
+    return {"blas": blas, "blas_threads": blas_threads(), "affinity_cores": affinity}
+
+
 def sample_rows_for(w: synth.Workload, target_s: float = 15.0) -> int:
     # oracle cost per row ~ 3 * 2 d V fp64 flops (logits, dHidden, dW) plus O(V) elementwise work
     per_row = 6.0 * w.d * w.V / 2.0e11 + w.V * 2.0e-7
@@ -264,11 +279,14 @@ def run_reference(args, w: synth.Workload, N: int):
     for i in range(args.warmup):
         oracle_sample(x, rows, seed=1000 + i)
     times = []
+    done = 0
     for i in range(args.steps):
         n, dt = oracle_sample(x, rows, seed=2000 + i)
         times.append(dt)
+        done += n
+    rows = done // max(1, args.steps)      # the sample never exceeds the workload's N rows
     total = sum(times)
-    value = rows * args.steps / total
+    value = done / total
     cores = blas_threads()
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1000.0 * total / args.steps, "higher_is_better": True,
@@ -278,7 +296,8 @@ def run_reference(args, w: synth.Workload, N: int):
                        "sample_rows_per_step": rows},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": f"{rows} seeded rows of the {w.name} workload per step, full fwd+bwd "
-                                       f"(loss, lse, dHidden, dW contribution) in numpy float64"},
+                                       f"(loss, lse, dHidden, dW contribution) in numpy float64",
+                             **host_cpu_info()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -480,7 +499,8 @@ def main_gpu(args, w: synth.Workload, N: int):
             n_rows, dt = oracle_sample(x, rows, seed=4242)
             cpu = {"value": n_rows / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                    "sample": f"{n_rows} seeded rows of the {w.name} workload, one full fwd+bwd "
-                             f"(loss, lse, dHidden, dW contribution) in numpy float64, {dt:.1f} s"}
+                             f"(loss, lse, dHidden, dW contribution) in numpy float64, {dt:.1f} s",
+                   **host_cpu_info()}
         bwd_plan = K.kdkl_backward_plan(Nn, d, V, Kc, args.chunk_tokens)
         out = {
             "metric": METRIC, "value": Nn * world / (ms_max * 1e-3), "unit": UNIT, "n_gpus": world,

@@ -1,10 +1,15 @@
-"""The multi-rank plumbing of bench.py on CPU with gloo (world size 2).
+"""The multi-rank plumbing of bench.py on CPU, and its reference arm.
 
-With N > 1 every rank runs an independent replica (different seeded batch)
-and the reported time is the slowest rank's; no collective touches the data.
+With N > 1 each rank draws its own seeded batch (its shard of the global
+batch of the token-sharded data-parallel step, whose collectives are tested in
+test_dp_orchestration.py and test_gpu_dp_ranks.py), and the reported time is
+the slowest rank's (max over ranks, gloo world size 2 here).
 """
+import json
 import os
 import socket
+import subprocess
+import sys
 
 import pytest
 import torch
@@ -13,6 +18,8 @@ import torch.multiprocessing as mp
 
 import bench
 import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def _free_port():
@@ -61,3 +68,15 @@ def test_reference_arm_prints_contract_line(steps, capsys, monkeypatch):
     assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["higher_is_better"] is True
+
+
+def test_reference_arm_counts_the_rows_it_times():
+    """The oracle sample never exceeds the workload's N rows, and the rate is computed from
+    the rows actually processed (the tiny workload has 256)."""
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "tiny",
+                          "--steps", "2", "--warmup", "0"], capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert out.returncode == 0, out.stderr
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    assert line["config"]["sample_rows_per_step"] == 256
+    assert line["cpu_baseline"]["sample"].startswith("256 seeded rows")
+    assert abs(line["value"] - 256 * 2 / (line["ms_per_step"] * 2 / 1000.0)) <= 1e-6 * line["value"]
