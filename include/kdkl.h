@@ -10,6 +10,8 @@
  * projection into the KL computation and never holds the full
  * [tokens x vocabulary] logit matrix; the backward recomputes each chunk's
  * projection (mind-verse.de article, three-variant list, "Fused chunked KL").
+ * kdkl_forward_backward computes the same outputs in one call, keeping each
+ * chunk's logits for that chunk's gradient instead of recomputing them.
  *
  * Definitions (N tokens, hidden size d, vocabulary V, K cached entries, tau):
  *   z[n, v]   = sum_j hidden[n, j] * W[v, j]              (student logits)
@@ -73,9 +75,11 @@ enum {
  * Bytes of scratch that kdkl_forward / kdkl_backward need for these sizes.
  * The amount is linear in N plus one N-independent chunk buffer of
  * chunk_tokens x V bf16 values (the backward's per-chunk logit gradient); it
- * never holds an N x V buffer.  chunk_tokens = 0 picks the library default
- * (min(N rounded up to 128, 8192)); other values are rounded up to a multiple
- * of 128.  Returns 0 for sizes that the entry points would reject.
+ * never holds an N x V buffer.  chunk_tokens = 0 sizes that buffer for the
+ * library's default capacity, min(N rounded up to 128, 8192) tokens, within
+ * which the backward's planner picks its chunk (kdkl_backward_plan); other
+ * values are rounded up to a multiple of 128 and used as given.  Returns 0 for
+ * sizes that the entry points would reject.
  */
 size_t kdkl_workspace_bytes(int64_t N, int32_t d, int32_t V, int32_t K, int64_t chunk_tokens);
 
