@@ -7,8 +7,9 @@ library; the only thing both sides see is the seeded input arrays.
 
 What it computes is the plain definition, written out without any of the
 kernel's blocking or fusion (the pages call the dense, forward-chunked and
-fused variants mathematically equivalent: mind-verse.de article, section "Ein
-zusammengefuehrter, chunked KL-Verlust", the three-variant list):
+fused variants mathematically equivalent: mind-verse.de article, section
+"Zwei systemische Optimierungen für Kosteneffizienz", item 2 "Ein
+zusammengeführter, chunked KL-Verlust", the three-variant list):
 
 * the student distribution P_S = softmax(z) with z = hidden @ W^T over the full
   vocabulary (the fused variant folds this output projection into the loss,
