@@ -21,6 +21,8 @@
 #include <cfloat>
 #include <cmath>
 
+#include <atomic>
+
 #include "kdkl_internal.h"
 #include "sm100.cuh"
 
@@ -900,12 +902,17 @@ template <int KIND, int BN, bool PAIR>
 static cudaError_t launch_one(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmOut,
                               const Sched& sc, const EpiParams& ep, int grid, cudaStream_t stream) {
   using C = GemmCfg<KIND, BN, PAIR>;
-  static bool configured = false;
-  if (!configured) {
-    const cudaError_t e = cudaFuncSetAttribute(gemm_kernel<KIND, BN, PAIR>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  // the dynamic shared-memory limit is a per-device attribute: set it on the first
+  // launch on each device (devices past the 64th get it on every launch)
+  static std::atomic<uint64_t> configured{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+  if (bit == 0 || !(configured.load(std::memory_order_acquire) & bit)) {
+    e = cudaFuncSetAttribute(gemm_kernel<KIND, BN, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return e;
-    configured = true;
+    configured.fetch_or(bit, std::memory_order_acq_rel);
   }
   if (PAIR) {
     cudaLaunchConfig_t cfg = {};
