@@ -226,15 +226,33 @@ def same_gpu_gemm_reference(dev, seconds: float = 3.0, size: int = 8192):
 
 
 # ----------------------------------------------------------------------------- oracle arm
-def oracle_sample(x: synth.Inputs, rows: int, seed: int):
-    """Times the CPU oracle (as it stands) on a bounded sample of the workload's rows."""
+# Rows per timed oracle sample, the same in the GPU line's cpu_baseline and in the
+# reference arm: one block of the oracle's row loop (its default row chunk), so the
+# two legs time identical work per sample.
+CPU_SAMPLE_ROWS = 64
+
+
+def oracle_weight(x: synth.Inputs):
+    """W widened to float64 once, outside every timed region (input marshalling, not the method)."""
+    from oracle import kl as O
+    return O.bf16_bits_to_f64(x.W_bits)
+
+
+def oracle_sample(x: synth.Inputs, W64, rows: int, seed: int):
+    """Times the CPU oracle (as it stands) on a bounded seeded sample of the workload's rows:
+    a full forward + backward of that sample (loss, lse, dHidden and its dW contribution)."""
     from oracle import kl as O
     sel = synth.sample_rows(x.hidden_bits.shape[0], rows, seed)
     sub = (x.hidden_bits[sel], x.W_bits, x.topk_idx[sel], x.topk_logit[sel], x.mask[sel], x.tau)
     t0 = time.perf_counter()
-    O.kl_loss(*sub)
+    O.kl_loss(*sub, W_f64=W64)
     dt = time.perf_counter() - t0
     return sel.size, dt
+
+
+def sample_text(rows: int, w: synth.Workload) -> str:
+    return (f"{rows} seeded rows of the {w.name} workload per sample, one full fwd+bwd (loss, lse, dHidden, "
+            f"dW contribution) in numpy float64; W widened to float64 once before timing")
 
 
 def blas_threads() -> int:
@@ -264,10 +282,17 @@ def host_cpu_info() -> dict:
     return {"blas": blas, "blas_threads": blas_threads(), "affinity_cores": affinity}
 
 
-def sample_rows_for(w: synth.Workload, target_s: float = 15.0) -> int:
-    # oracle cost per row ~ 3 * 2 d V fp64 flops (logits, dHidden, dW) plus O(V) elementwise work
-    per_row = 6.0 * w.d * w.V / 2.0e11 + w.V * 2.0e-7
-    return int(max(16, min(4096, target_s / per_row)))
+def cpu_baseline(x: synth.Inputs, w: synth.Workload, W64, budget_s: float = 8.0, max_samples: int = 16):
+    """The oracle timed on repeated seeded samples of CPU_SAMPLE_ROWS rows (about budget_s seconds)."""
+    done, total, i = 0, 0.0, 0
+    while i < max_samples and (i < 2 or total < budget_s):
+        n, dt = oracle_sample(x, W64, CPU_SAMPLE_ROWS, seed=4242 + i)
+        done += n
+        total += dt
+        i += 1
+    return {"value": done / total, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": sample_text(min(CPU_SAMPLE_ROWS, x.hidden_bits.shape[0]), w) + f"; {i} samples, {total:.1f} s",
+            **host_cpu_info()}
 
 
 def run_reference(args, w: synth.Workload, N: int):
@@ -275,13 +300,13 @@ def run_reference(args, w: synth.Workload, N: int):
     if rank != 0:
         return 0
     x = synth.make_inputs(w, N=N)
-    rows = sample_rows_for(w, target_s=max(2.0, 60.0 / max(1, args.steps + args.warmup)))
+    W64 = oracle_weight(x)
     for i in range(args.warmup):
-        oracle_sample(x, rows, seed=1000 + i)
+        oracle_sample(x, W64, CPU_SAMPLE_ROWS, seed=1000 + i)
     times = []
     done = 0
     for i in range(args.steps):
-        n, dt = oracle_sample(x, rows, seed=2000 + i)
+        n, dt = oracle_sample(x, W64, CPU_SAMPLE_ROWS, seed=2000 + i)
         times.append(dt)
         done += n
     rows = done // max(1, args.steps)      # the sample never exceeds the workload's N rows
@@ -295,9 +320,7 @@ def run_reference(args, w: synth.Workload, N: int):
             "config": {"workload": w.name, "N": N, "d": w.d, "V": w.V, "K": w.K, "tau": w.tau,
                        "sample_rows_per_step": rows},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": f"{rows} seeded rows of the {w.name} workload per step, full fwd+bwd "
-                                       f"(loss, lse, dHidden, dW contribution) in numpy float64",
-                             **host_cpu_info()},
+                             "sample": sample_text(rows, w), **host_cpu_info()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -320,6 +343,108 @@ def max_over_ranks(value: float, device, world: int) -> float:
 
 
 # ----------------------------------------------------------------------------- GPU arm
+def _bf16(bits):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+
+
+def time_workload(K, dev, x: synth.Inputs, *, fused: bool, steps: int, warmup: int, chunk_tokens: int = 0):
+    """Forward + backward (or the fused step) on device-resident inputs: warm-up steps,
+    then `steps` steps timed with CUDA events on the launching stream, with the clocks
+    sampled meanwhile and the peak of torch-allocated bytes (inputs, outputs, workspace)."""
+    import torch
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
+    base = torch.cuda.memory_allocated(dev)
+    torch.cuda.reset_peak_memory_stats(dev)
+    Nn, d, V, Kc = x.shape
+    hidden, W = _bf16(x.hidden_bits).to(dev), _bf16(x.W_bits).to(dev)
+    idx, logit = torch.from_numpy(x.topk_idx).to(dev), torch.from_numpy(x.topk_logit).to(dev)
+    mask = torch.from_numpy(x.mask).to(dev)
+    ws_bytes = (K.kdkl_forward_backward_workspace_bytes(Nn, d, V, Kc, chunk_tokens) if fused
+                else K.kdkl_workspace_bytes(Nn, d, V, Kc, chunk_tokens))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    lse = torch.empty(Nn, dtype=torch.float32, device=dev)
+    dH = torch.empty(Nn, d, dtype=torch.bfloat16, device=dev)
+    dW = torch.empty(V, d, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        if fused:
+            K.kdkl_forward_backward(hidden, W, idx, logit, mask, x.tau, loss, lse, dH, dW, ws,
+                                    chunk_tokens=chunk_tokens, stream=stream)
+        else:
+            K.kdkl_forward(hidden, W, idx, logit, mask, x.tau, loss, lse, ws, stream=stream)
+            K.kdkl_backward(hidden, W, idx, logit, mask, x.tau, lse, None, dH, dW, ws, chunk_tokens=chunk_tokens,
+                            stream=stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    flags = K.kdkl_read_device_flags(ws)
+    peak = torch.cuda.max_memory_allocated(dev) - base
+    sampler = ClockSampler(gpu_id_for(dev.index or 0))
+    sampler.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1) / steps
+    del hidden, W, idx, logit, mask, ws, loss, lse, dH, dW
+    torch.cuda.empty_cache()
+    flops = (6.0 if fused else 8.0) * Nn * d * V
+    return {"N": Nn, "ms_per_step": ms, "tokens_per_s": Nn / (ms * 1e-3),
+            "tflops": synth.flops_fwd_bwd(Nn, d, V) / (ms * 1e-3) / 1e12,
+            "executed_tflops": flops / (ms * 1e-3) / 1e12, "peak_gb": peak / 1e9, "workspace_gb": ws_bytes / 1e9,
+            "device_flags": flags, "steps": steps, "warmup": warmup,
+            "sm_mhz": clocks.get("sm_mhz"), "clock_reasons": clocks.get("reasons")}
+
+
+def extra_workloads(K, dev, peaks, steps: int = 2, warmup: int = 3) -> dict:
+    """The metric's other parts on the same run: peak memory and throughput against N over
+    the long-context sweep (one seeded draw at the largest N, leading rows for the smaller
+    N), the large-vocabulary head, and the one-call fused step on the 8B-class head."""
+    out = {}
+    t0 = time.perf_counter()
+    sw = synth.CONFIGS["sweep"]
+    big = synth.make_inputs(sw, N=max(synth.SWEEP_N))
+    pts = []
+    for n in synth.SWEEP_N:
+        sub = synth.Inputs(big.hidden_bits[:n], big.W_bits, big.topk_idx[:n], big.topk_logit[:n], big.mask[:n],
+                           big.tau)
+        r = time_workload(K, dev, sub, fused=False, steps=steps, warmup=warmup)
+        r["frac_of_bf16_peak"] = r["tflops"] / peaks["bf16_tflops"]
+        pts.append(r)
+    del big
+    # peak = a + b N over the points whose chunk buffer has its full 8192-token size
+    fit_pts = [p for p in pts if p["N"] >= 16384]
+    Ns = np.array([p["N"] for p in fit_pts], dtype=float)
+    P = np.array([p["peak_gb"] * 1e9 for p in fit_pts])
+    b, a = np.polyfit(Ns, P, 1)
+    out["sweep"] = {"workload": f"sweep d={sw.d} V={sw.V} K={sw.K} tau={sw.tau}",
+                    "inputs": f"one seeded draw at N={max(synth.SWEEP_N)}, leading rows for smaller N",
+                    "points": pts,
+                    "peak_fit": {"over_N": [int(n) for n in Ns], "intercept_gb": a / 1e9,
+                                 "slope_kb_per_token": b / 1e3, "max_resid_mb": float(np.abs(P - a - b * Ns).max()) / 1e6,
+                                 "nxv_bf16_kb_per_token": 2 * sw.V / 1e3}}
+    lv = synth.CONFIGS["large_vocab"]
+    r = time_workload(K, dev, synth.make_inputs(lv), fused=False, steps=steps, warmup=warmup)
+    r["frac_of_bf16_peak"] = r["tflops"] / peaks["bf16_tflops"]
+    r["frac_of_bf16_peak_sustained"] = r["tflops"] / peaks["bf16_tflops_sustained"]
+    out["large_vocab"] = r
+    w8 = synth.CONFIGS["8b"]
+    r = time_workload(K, dev, synth.make_inputs(w8), fused=True, steps=max(steps, 3), warmup=warmup)
+    r["note"] = "kdkl_forward_backward: each chunk's logits computed once (6 N d V executed); tflops counts 8 N d V"
+    out["fused_step_8b"] = r
+    out["extras_wall_s"] = time.perf_counter() - t0
+    return out
+
+
 def main_gpu(args, w: synth.Workload, N: int):
     import torch
     import torch.distributed as dist
@@ -341,17 +466,14 @@ def main_gpu(args, w: synth.Workload, N: int):
     t_gen = time.perf_counter() - t_gen
     Nn, d, V, Kc = x.shape
 
-    def bf16(bits):
-        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
-
-    h_hidden = bf16(x.hidden_bits).pin_memory()
+    h_hidden = _bf16(x.hidden_bits).pin_memory()
     h_idx = torch.from_numpy(x.topk_idx).pin_memory()
     h_logit = torch.from_numpy(x.topk_logit).pin_memory()
     h_mask = torch.from_numpy(x.mask).pin_memory()
     torch.cuda.synchronize()
     torch.cuda.reset_peak_memory_stats(dev)
     base_alloc = torch.cuda.memory_allocated(dev)
-    W = bf16(x.W_bits).to(dev)
+    W = _bf16(x.W_bits).to(dev)
     if world > 1:
         dist.broadcast(W, src=0)     # one output-head weight, replicated (data parallelism)
 
@@ -370,11 +492,13 @@ def main_gpu(args, w: synth.Workload, N: int):
     dW = torch.empty(V, d, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    # N > 1: token-sharded data parallelism (output_head_kl_b200.dp): each rank's
-    # batch is its shard, the loss normaliser is the all-reduced valid count and
-    # dW is all-reduced (sum) over NCCL, the step's one real exchange.
+    # N > 1: token-sharded data parallelism (output_head_kl_b200.dp): each rank's batch
+    # is its shard; the library counts the shard's valid tokens, the counts are summed
+    # over NCCL, forward and backward normalise by that sum, the per-rank losses are
+    # summed and dW is all-reduced (sum), the step's one real exchange.
     n_total = torch.zeros(1, dtype=torch.int32, device=dev)
     dp_opts = K.kdkl_options(n_valid_global=n_total) if world > 1 else None
+    n_local = K.n_valid_view(ws) if world > 1 else None
 
     def step(bufs=None):
         hidden_, idx_, logit_, mask_ = bufs if bufs is not None else (hidden, idx, logit, mask)
@@ -382,14 +506,17 @@ def main_gpu(args, w: synth.Workload, N: int):
             K.kdkl_forward_backward(hidden_, W, idx_, logit_, mask_, x.tau, loss, lse, dH, dW, ws,
                                     chunk_tokens=args.chunk_tokens, stream=stream)
             return
-        K.kdkl_forward(hidden_, W, idx_, logit_, mask_, x.tau, loss, lse, ws, stream=stream)
         if world > 1:
-            n_total.copy_(ws[4:8].view(torch.int32))
+            K.kdkl_count_valid(idx_, logit_, mask_, x.tau, V, ws, dp_opts, stream=stream)
+            n_total.copy_(n_local)
             dist.all_reduce(n_total)
+            K.kdkl_forward_ex(hidden_, W, idx_, logit_, mask_, x.tau, loss, lse, ws, dp_opts, stream=stream)
+            dist.all_reduce(loss)
             K.kdkl_backward_ex(hidden_, W, idx_, logit_, mask_, x.tau, lse, None, dH, dW, ws, dp_opts,
                                chunk_tokens=args.chunk_tokens, stream=stream)
             dist.all_reduce(dW)
         else:
+            K.kdkl_forward(hidden_, W, idx_, logit_, mask_, x.tau, loss, lse, ws, stream=stream)
             K.kdkl_backward(hidden_, W, idx_, logit_, mask_, x.tau, lse, None, dH, dW, ws,
                             chunk_tokens=args.chunk_tokens, stream=stream)
 
@@ -469,6 +596,7 @@ def main_gpu(args, w: synth.Workload, N: int):
 
     out = None
     ref_gemm = None
+    extras = None
     if rank == 0 and not args.no_gemm_reference:
         ref_gemm = same_gpu_gemm_reference(dev)
     if rank == 0:
@@ -495,12 +623,7 @@ def main_gpu(args, w: synth.Workload, N: int):
         kernels = {k: {"launches": v[0], "ms_per_step": v[1] / args.steps} for k, v in kt.items() if v[0]}
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            rows = sample_rows_for(w)
-            n_rows, dt = oracle_sample(x, rows, seed=4242)
-            cpu = {"value": n_rows / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-                   "sample": f"{n_rows} seeded rows of the {w.name} workload, one full fwd+bwd "
-                             f"(loss, lse, dHidden, dW contribution) in numpy float64, {dt:.1f} s",
-                   **host_cpu_info()}
+            cpu = cpu_baseline(x, w, oracle_weight(x))
         bwd_plan = K.kdkl_backward_plan(Nn, d, V, Kc, args.chunk_tokens)
         out = {
             "metric": METRIC, "value": Nn * world / (ms_max * 1e-3), "unit": UNIT, "n_gpus": world,
@@ -512,7 +635,10 @@ def main_gpu(args, w: synth.Workload, N: int):
                        "parallelism": f"dp{world}" if world > 1 else "single",
                        "schedule": ("fused step: each chunk's logits computed once and kept for its gradient "
                                     "(6 N d V flops executed)") if args.fused_step else
-                                   "kdkl_forward + kdkl_backward (the backward recomputes each chunk's logits)"},
+                                   "kdkl_forward + kdkl_backward (the backward recomputes each chunk's logits)",
+                       "e2e": "per step: the batch (hidden, topk_idx, topk_logit, mask) copied host->device from "
+                              "pinned memory and the loss read back; W stays resident as a model weight, and "
+                              "dHidden and dW stay on the device for the optimizer and the layers below"},
             "tflops": tflops,
             "frac_of_bf16_peak": tflops / peaks["bf16_tflops"],
             "frac_of_bf16_peak_sustained": tflops / peaks["bf16_tflops_sustained"],
@@ -532,10 +658,16 @@ def main_gpu(args, w: synth.Workload, N: int):
             "device_flags": flags,
             "input_gen_s": t_gen,
         }
-        print(json.dumps(out), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+    elif out is not None and not args.no_extras and not args.fused_step and w.name == "8b":
+        del hidden, idx, logit, mask, ws, loss, lse, dH, dW, W, h_hidden, h_idx, h_logit, h_mask
+        torch.cuda.empty_cache()
+        extras = extra_workloads(K, dev, measured_peaks())
+        out.update(extras)
+    if out is not None:
+        print(json.dumps(out), flush=True)
     return 0
 
 
@@ -602,6 +734,8 @@ def main():
     ap.add_argument("--N", type=int, default=None, help="token count override (sweep points)")
     ap.add_argument("--chunk-tokens", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the sweep, large-vocabulary and fused-step objects of the default line")
     ap.add_argument("--no-gemm-reference", action="store_true",
                     help="skip the same-GPU cuBLAS GEMM timed after the run (context only)")
     ap.add_argument("--topk", action="store_true", help="time the teacher top-K cache producer instead")
@@ -624,6 +758,7 @@ def main():
     if args.sweep:
         args.no_cpu_baseline = True
         args.no_gemm_reference = True
+        args.no_extras = True
         for n in synth.SWEEP_N:
             rc = main_gpu(args, synth.CONFIGS["sweep"], n)
             if rc:

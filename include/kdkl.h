@@ -68,7 +68,11 @@ enum {
   KDKL_DEV_IDX_RANGE = 1u, /* some cached index was outside [0, V); the entry was dropped */
   KDKL_DEV_IDX_DUP = 2u,   /* some row repeated a cached index; the probabilities were added */
   KDKL_DEV_NONFINITE = 4u, /* some row had a NaN/+inf (or only -inf) logit; the row was masked */
-  KDKL_DEV_TIMEOUT = 8u    /* an internal pipeline wait gave up; this call's outputs are invalid */
+  KDKL_DEV_TIMEOUT = 8u,   /* an internal pipeline wait gave up (after 2 s): the kernel stopped early,
+                              so this call's outputs, and those of every later call on the stream
+                              that read them, are invalid */
+  KDKL_DEV_BOUNDS = 16u    /* bounds-checking build (libkdkl_debug.so) only: an index check in a
+                              kernel failed and the access was skipped; outputs are invalid */
 };
 
 /*
@@ -139,7 +143,8 @@ kdkl_status kdkl_backward(const void* hidden, const void* W, const int32_t* topk
  *     fit at K = 100.
  *   - The first call on each device looks up that device's copy of the array
  *     (cudaGetSymbolAddress) with the device current; make that first call
- *     before any stream capture.
+ *     before any stream capture.  The lookup is kept per device and CUDA
+ *     context: after cudaDeviceReset the next call looks the array up again.
  *   - Every call on a device shares the one array and leaves its contents
  *     behind.  Each call clears what must start at zero, so leftovers do not
  *     matter, but two calls that overlap on the GPU (other streams, other host
@@ -180,9 +185,10 @@ typedef struct {
   int32_t kd_scale_tau_sq;  /* nonzero: multiply the KL term by student_tau^2 (default 0) */
   float ce_weight;          /* finite, >= 0 (default 0: no hard-label term) */
   const int32_t* labels;    /* [N] int32 device, 4-byte aligned; required when ce_weight > 0 */
-  /* Data-parallel normaliser: a device count to divide by instead of this
-   * call's own N_valid (e.g. the sum of every rank's kdkl_n_valid_device count
-   * after an all-reduce).  NULL = this call's own count (default). */
+  /* Data-parallel normaliser: a device count to divide the loss and the
+   * gradients by instead of this call's own N_valid (the sum over ranks of each
+   * rank's kdkl_count_valid count, after an all-reduce).  NULL = this call's own
+   * count (default).  Forward and backward must get the same count. */
   const uint32_t* n_valid_global;
   /* N tile width of the backward's dHidden and dW GEMMs (their N axis is d):
    * 0 = the planner's choice (default; see kdkl_backward_plan), else one of
@@ -194,9 +200,31 @@ typedef struct {
 
 void kdkl_options_init(kdkl_options* options);
 
-/* Device address of the N_valid count that the last forward/backward on this
- * workspace computed (uint32, stream-ordered after that call; no CUDA call is made). */
+/* Device address of the N_valid count that the last kdkl_count_valid, forward or
+ * backward call on this workspace computed: this call's own rows, even when
+ * options->n_valid_global was given (uint32, stream-ordered after that call; no CUDA
+ * call is made; NULL when workspace is NULL). */
 const uint32_t* kdkl_n_valid_device(const void* workspace);
+
+/*
+ * Count of the rows that enter the loss, without the projection: runs the
+ * forward's per-row preparation of the teacher cache (the mask, dropped and
+ * non-finite entries; see the data-error rules above) and leaves the count at
+ * kdkl_n_valid_device(workspace) and the data-error flags in the flag word.
+ * It exists for data parallelism (the paper's training runs shard tokens across
+ * GPUs): each rank counts its own shard, the counts are summed across ranks on
+ * the device (an all-reduce), and the sum is passed as options->n_valid_global
+ * to kdkl_forward_ex and kdkl_backward_ex.  Each rank's loss is then its rows'
+ * share of the global loss (the sum over ranks is the global loss), its dHidden
+ * is final, and its dW is its term of the global dW.
+ *   topk_idx, topk_logit, mask, N, V, K, tau, options: as kdkl_forward_ex
+ *   workspace >= kdkl_workspace_bytes(N, d, V, K, c) for any d and c, 256-byte
+ *     aligned; the same workspace may then be passed to the forward and backward
+ * N = 0 leaves a count of 0.
+ */
+kdkl_status kdkl_count_valid(const void* topk_idx, const void* topk_logit, const uint8_t* mask, int64_t N,
+                             int32_t V, int32_t K, float tau, const kdkl_options* options, void* workspace,
+                             size_t workspace_bytes, void* stream);
 
 /* kdkl_forward with options (NULL = defaults); topk_idx / topk_logit typed by options->cache_format. */
 kdkl_status kdkl_forward_ex(const void* hidden, const void* W, const void* topk_idx, const void* topk_logit,

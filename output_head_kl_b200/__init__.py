@@ -7,7 +7,7 @@ raises.
 
 Names mirror the C entry points: ``kdkl_workspace_bytes``, ``kdkl_forward``,
 ``kdkl_backward``, ``kdkl_forward_ex``, ``kdkl_backward_ex`` (with ``kdkl_options``),
-``kdkl_forward_noalloc``, ``kdkl_teacher_topk``, ``kdkl_read_device_flags``, ``kdkl_timing_enable``,
+``kdkl_forward_noalloc``, ``kdkl_teacher_topk``, ``kdkl_count_valid``, ``kdkl_read_device_flags``, ``kdkl_timing_enable``,
 ``kdkl_timing_read``, ``kdkl_status_string``, ``kdkl_last_error``.  ``fused_kl_forward_backward`` is a convenience wrapper
 that allocates the outputs and the workspace with torch (the library itself
 never allocates).
@@ -19,11 +19,13 @@ import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "_lib", "libkdkl.so")
+# The same library with in-kernel index checks (KDKL_DEV_BOUNDS); see build.py.
+DEBUG_LIB_PATH = os.path.join(_HERE, "_lib", "libkdkl_debug.so")
 
 KDKL_OK = 0
 STATUS_NAMES = {0: "KDKL_OK", 1: "KDKL_ERR_NULL", 2: "KDKL_ERR_SHAPE", 3: "KDKL_ERR_ALIGN",
                 4: "KDKL_ERR_UNSUPPORTED", 5: "KDKL_ERR_WORKSPACE", 6: "KDKL_ERR_CUDA"}
-DEV_IDX_RANGE, DEV_IDX_DUP, DEV_NONFINITE, DEV_TIMEOUT = 1, 2, 4, 8
+DEV_IDX_RANGE, DEV_IDX_DUP, DEV_NONFINITE, DEV_TIMEOUT, DEV_BOUNDS = 1, 2, 4, 8, 16
 
 _lib = None
 
@@ -106,6 +108,8 @@ def lib() -> ctypes.CDLL:
     L.kdkl_teacher_topk.restype = ctypes.c_int
     L.kdkl_n_valid_device.argtypes = [vp]
     L.kdkl_n_valid_device.restype = ctypes.c_void_p
+    L.kdkl_count_valid.argtypes = [vp, vp, vp, i64, i32, i32, f32, ctypes.POINTER(Options), vp, sz, vp]
+    L.kdkl_count_valid.restype = ctypes.c_int
     L.kdkl_selftest_wait_timeout.argtypes = [vp, ctypes.c_uint64, vp]
     L.kdkl_selftest_wait_timeout.restype = ctypes.c_int
     L.kdkl_timing_enable.argtypes = [ctypes.c_int]
@@ -297,6 +301,30 @@ def kdkl_forward_noalloc(hidden, W, topk_idx, topk_logit, mask, tau, loss, lse, 
 def kdkl_n_valid_device(workspace) -> int:
     """Device address of the workspace's N_valid count (uint32)."""
     return int(lib().kdkl_n_valid_device(_ptr(workspace)))
+
+
+def n_valid_view(workspace):
+    """A one-element int32 view of the workspace tensor (uint8) at the address
+    kdkl_n_valid_device returns (the count fits 31 bits: N is at most 2^31 - 256)."""
+    import torch
+    off = kdkl_n_valid_device(workspace) - workspace.data_ptr()
+    if not 0 <= off <= workspace.numel() * workspace.element_size() - 4 or off % 4:
+        raise RuntimeError(f"kdkl_n_valid_device gave an offset {off} outside the workspace")
+    return workspace.view(torch.uint8)[off:off + 4].view(torch.int32)
+
+
+def kdkl_count_valid(topk_idx, topk_logit, mask, tau, V, workspace, options=None, *, N=None, K=None,
+                     workspace_bytes=None, stream=None, check=True) -> int:
+    """Calls kdkl_count_valid: this shard's valid-token count, left at kdkl_n_valid_device(workspace)."""
+    N = topk_idx.shape[0] if N is None else N
+    K = topk_idx.shape[1] if K is None else K
+    wsb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    opt = ctypes.byref(options) if options is not None else None
+    st = lib().kdkl_count_valid(_ptr(topk_idx), _ptr(topk_logit), _ptr(mask), int(N), int(V), int(K), float(tau),
+                                opt, _ptr(workspace), int(wsb), _stream(stream))
+    if check:
+        _check(st, "kdkl_count_valid")
+    return st
 
 
 def kdkl_read_device_flags(workspace, stream=None) -> int:

@@ -2,6 +2,13 @@
 
 Every kernel is compiled for sm_100a only.  Run ``python -m output_head_kl_b200.build``
 (or ``__graft_entry__.build()``); the result travels with the source tree.
+
+A second library, ``_lib/libkdkl_debug.so``, is the same sources compiled with
+``-DKDKL_DEBUG``: every list walk, partial-result slot, shared-memory list write,
+TMA coordinate and lockstep slot is range-checked in the kernels, and a failed
+check sets ``KDKL_DEV_BOUNDS`` in the device flag word and skips (or clamps) the
+access instead of making it.  It stands in for a memory checker, which this
+hardware pool does not offer; the tests run the ragged parity cases through it.
 """
 from __future__ import annotations
 
@@ -14,6 +21,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 OUT_DIR = os.path.join(HERE, "_lib")
 LIB = os.path.join(OUT_DIR, "libkdkl.so")
+DEBUG_LIB = os.path.join(OUT_DIR, "libkdkl_debug.so")
 SOURCES = ("kernels.cu", "api.cu", "noalloc.cu")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
@@ -27,41 +35,48 @@ def nvcc() -> str:
     return path
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, f) for f in os.listdir(CSRC)]
     deps.append(os.path.join(os.path.dirname(HERE), "include", "kdkl.h"))
     deps.append(os.path.abspath(__file__))
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
-        return LIB
-    os.makedirs(OUT_DIR, exist_ok=True)
+def _build_one(lib: str, prefix: str, defines, log_name: str):
     objs = []
     logs = []
     for src in SOURCES:
-        obj = os.path.join(OUT_DIR, src.replace(".cu", ".o"))
-        cmd = [nvcc(), *ARCH, *FLAGS, "-I", os.path.join(os.path.dirname(HERE), "include"), "-c",
+        obj = os.path.join(OUT_DIR, prefix + src.replace(".cu", ".o"))
+        cmd = [nvcc(), *ARCH, *FLAGS, *defines, "-I", os.path.join(os.path.dirname(HERE), "include"), "-c",
                os.path.join(CSRC, src), "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         logs.append(r.stdout + r.stderr)
         if r.returncode != 0:
             raise RuntimeError(f"nvcc failed on {src}:\n{r.stdout}\n{r.stderr}")
         objs.append(obj)
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *objs]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    with open(os.path.join(OUT_DIR, "ptxas.log"), "w") as f:
+    os.replace(tmp, lib)
+    with open(os.path.join(OUT_DIR, log_name), "w") as f:
         f.write("\n".join(logs))
-    if verbose:
-        print("\n".join(logs))
+    return logs
+
+
+def build(force: bool = False, verbose: bool = False, debug: bool = True) -> str:
+    """Builds libkdkl.so (and, with debug=True, the bounds-checking libkdkl_debug.so)."""
+    os.makedirs(OUT_DIR, exist_ok=True)
+    if force or _stale(LIB):
+        logs = _build_one(LIB, "", [], "ptxas.log")
+        if verbose:
+            print("\n".join(logs))
+    if debug and (force or _stale(DEBUG_LIB)):
+        _build_one(DEBUG_LIB, "dbg_", ["-DKDKL_DEBUG"], "ptxas_debug.log")
     return LIB
 
 

@@ -13,6 +13,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -43,6 +44,7 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 constexpr int64_t kDefaultChunk = 8192;
+constexpr int kDefaultSyncWindow = 4;
 constexpr int64_t kMaxRows = (int64_t(1) << 31) - 256;
 constexpr int32_t kMaxV = (int32_t(1) << 30);
 
@@ -437,6 +439,45 @@ EpiParams base_params(const Common& c, const WsLayout& L) {
   return ep;
 }
 
+// Tiles a group may run ahead of the slowest group sharing its vocabulary split
+// (the lockstep of the row-stream GEMMs; 0 = off).  KDKL_SYNC_WINDOW overrides the
+// default, for tuning.
+int sync_window() {
+  static int w = [] {
+    const char* e = std::getenv("KDKL_SYNC_WINDOW");
+    int v = kDefaultSyncWindow;
+    if (e && *e) v = std::atoi(e);
+    return v < 0 ? 0 : v;
+  }();
+  return w;
+}
+
+// L2 eviction priorities of the operand loads (KDKL_L2_HINTS, a bit mask, for tuning;
+// default 0 = every load at normal priority):
+//   bit 0: the hidden rows of the row-stream GEMMs (each row block is re-read for every
+//          vocabulary tile of its unit) are kept with evict_last;
+//   bit 1: the dW GEMM's hidden chunk (re-read by every vocabulary row block) likewise.
+int l2_hint_mask() {
+  static int m = [] {
+    const char* e = std::getenv("KDKL_L2_HINTS");
+    return (e && *e) ? std::atoi(e) : 0;
+  }();
+  return m;
+}
+
+// Arms the lockstep of a row-stream launch of `grid` CTAs: clears the groups'
+// position words on the stream, ahead of the launch.
+cudaError_t arm_sync(Sched& sc, unsigned long long* prog, int grid, bool pair, cudaStream_t s) {
+  const int groups = pair ? grid / 2 : grid;
+  sc.sync_window = 0;
+  sc.prog = prog;
+  if (l2_hint_mask() & 1) sc.l2_a = kL2Last;
+  const int w = sync_window();
+  if (w <= 0 || groups > kSyncSlots || groups < 2) return cudaSuccess;
+  sc.sync_window = w;
+  return cudaMemsetAsync(prog, 0, static_cast<size_t>(groups) * 8, s);
+}
+
 }  // namespace
 
 WsLayout make_layout(int64_t N, int32_t d, int32_t V, int32_t K, int64_t chunk_tokens) {
@@ -455,6 +496,8 @@ WsLayout make_layout(int64_t N, int32_t d, int32_t V, int32_t K, int64_t chunk_t
   size_t off = 0;
   L.header = off;
   off += 256;
+  L.sync = off;
+  off += static_cast<size_t>(kSyncSlots) * 8;
   L.sidx = off;
   off = align_up(off + static_cast<size_t>(N) * L.Kp * 4, 256);
   L.sprob = off;
@@ -548,7 +591,10 @@ static kdkl_status forward_impl(const void* hidden, const void* W, const void* t
   ep.part_m = part;
   ep.part_s = part + plane;
   ep.part_a = part + 2 * plane;
+  ep.part_cap = static_cast<int64_t>(plane);
   const int grid = pr.grid(sc.units);
+  if ((e = arm_sync(sc, at<unsigned long long>(workspace, L.sync), grid, pr.pair, s)) != cudaSuccess)
+    return cuda_fail(e, "cudaMemsetAsync");
   if ((e = timed(kTFwd, s, [&] { return launch_gemm(kEpiLse, 256, pr.pair, tmA, tmB, tmA, sc, ep, grid, s); })) !=
       cudaSuccess)
     return cuda_fail(e, "forward GEMM launch");
@@ -557,7 +603,7 @@ static kdkl_status forward_impl(const void* hidden, const void* W, const void* t
          return launch_merge(ep.part_m, ep.part_s, ep.part_a, splits, pr.rows, c.opt.student_tau,
                              at<float>(workspace, L.negent), at<float>(workspace, L.wsum),
                              at<uint8_t>(workspace, L.rowmask), N, lse, loss, at<double>(workspace, L.blocksum),
-                             header, ep.n_valid, 0, 0, s);
+                             header, ep.n_valid, 0, 0, static_cast<int64_t>(plane), s);
        })) != cudaSuccess)
     return cuda_fail(e, "merge launch");
   return ok();
@@ -605,6 +651,7 @@ static kdkl_status run_dh_dw(const EpiParams& ep0, const Pairing& pd, int bn, in
   {
     const int64_t vb = (V + pd.rows - 1) / pd.rows;
     Sched sc{static_cast<int>(vb * nt), 1, nt, static_cast<int>((nc + kBK - 1) / kBK), 0};
+    if (l2_hint_mask() & 2) sc.l2_b = kL2Last;
     EpiParams ep = ep0;
     ep.M = V;
     ep.Ncols = d;
@@ -612,9 +659,14 @@ static kdkl_status run_dh_dw(const EpiParams& ep0, const Pairing& pd, int bn, in
     ep.dW = dW;
     ep.ldo = d;
     ep.accumulate = c0 > 0 ? 1 : 0;
+    // dW blocks of 32 rows x 32 fp32 columns, 128-byte swizzle: the epilogue's TMA loads
+    // of the old values and stores of the new ones
+    CUtensorMap tmDW;
+    if (!make_map_f32(&tmDW, dW, d, V, d, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+      return fail(KDKL_ERR_CUDA, "cuTensorMapEncodeTiled failed (dW)");
     const int grid = pd.grid(sc.units);
     if ((e = timed(kTDw, s, [&] {
-           return launch_gemm(kEpiRmwF32, bn, pd.pair, tmG_mn, tmH_mn, tmG_mn, sc, ep, grid, s);
+           return launch_gemm(kEpiRmwF32, bn, pd.pair, tmG_mn, tmH_mn, tmDW, sc, ep, grid, s);
          })) != cudaSuccess)
       return cuda_fail(e, "dW GEMM launch");
   }
@@ -685,6 +737,8 @@ static kdkl_status backward_impl(const void* hidden, const void* W, const void* 
       ep.Ncols = V;
       ep.row_offset = c0;
       const int grid = pg.grid(sc.units);
+      if ((e = arm_sync(sc, at<unsigned long long>(workspace, L.sync), grid, pg.pair, s)) != cudaSuccess)
+        return cuda_fail(e, "cudaMemsetAsync");
       if ((e = timed(kTGrad, s, [&] {
              return launch_gemm(kEpiGrad, 256, pg.pair, tmH_k, tmW_k, tmG_store, sc, ep, grid, s);
            })) != cudaSuccess)
@@ -790,7 +844,10 @@ static kdkl_status forward_backward_impl(const void* hidden, const void* W, cons
       ep.part_m = part;
       ep.part_s = part + plane;
       ep.part_a = part + 2 * plane;
+      ep.part_cap = static_cast<int64_t>(plane);
       const int grid = pg.grid(sc.units);
+      if ((e = arm_sync(sc, at<unsigned long long>(workspace, L.sync), grid, pg.pair, s)) != cudaSuccess)
+        return cuda_fail(e, "cudaMemsetAsync");
       if ((e = timed(kTFusedFwd, s, [&] {
              return launch_gemm(kEpiLseStore, 256, pg.pair, tmH_k, tmW_k, tmZ, sc, ep, grid, s);
            })) != cudaSuccess)
@@ -801,13 +858,14 @@ static kdkl_status forward_backward_impl(const void* hidden, const void* W, cons
            return launch_merge(part, part + plane, part + 2 * plane, splits, pg.rows, c.opt.student_tau,
                                at<float>(workspace, L.negent) + c0, at<float>(workspace, L.wsum) + c0,
                                at<uint8_t>(workspace, L.rowmask) + c0, nc, lse + c0, loss,
-                               at<double>(workspace, L.blocksum), header, ep0.n_valid, c0 / 256, total_blocks, s);
+                               at<double>(workspace, L.blocksum), header, ep0.n_valid, c0 / 256, total_blocks,
+                               static_cast<int64_t>(plane), s);
          })) != cudaSuccess)
       return cuda_fail(e, "merge launch");
     // (3) G from the stored logits
     if ((e = timed(kTGPass, s, [&] {
            return launch_gpass(zbuf, L.Vp, gbuf, L.Vp, nc, V, c0, ep0.sidx, ep0.sprob, ep0.Kp, ep0.rowmask,
-                               ep0.wsum, lse, ep0.n_valid, grad_loss, c.opt.student_tau, s);
+                               ep0.wsum, lse, ep0.n_valid, grad_loss, c.opt.student_tau, ep0.flags, s);
          })) != cudaSuccess)
       return cuda_fail(e, "G launch");
     // (4) dHidden rows of the chunk = G W; (5) dW (+)= G^T hidden_chunk
@@ -875,6 +933,36 @@ kdkl_status kdkl_backward_plan(int64_t N, int32_t d, int32_t V, int32_t K, int64
   return ok();
 }
 
+kdkl_status kdkl_count_valid(const void* topk_idx, const void* topk_logit, const uint8_t* mask, int64_t N,
+                             int32_t V, int32_t K, float tau, const kdkl_options* options, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  // the count needs no hidden states or weights; d only sizes the backward's buffers
+  const Common c{nullptr,   nullptr,   topk_idx,        topk_logit, mask, N, 8, V, K, tau,
+                 workspace, workspace_bytes, options ? *options : default_options()};
+  kdkl_status st = check_shapes(N, 8, V, K, tau);
+  if (st != KDKL_OK) return st;
+  if (!topk_idx || !topk_logit || !mask || !workspace)
+    return fail(KDKL_ERR_NULL, "topk_idx, topk_logit, mask and workspace must be non-NULL");
+  if ((st = check_options(c)) != KDKL_OK) return st;
+  const size_t cache_align = c.opt.cache_format == KDKL_CACHE_U16_BF16 ? 2 : 4;
+  if (!aligned(topk_idx, cache_align) || !aligned(topk_logit, cache_align))
+    return fail(KDKL_ERR_ALIGN, "topk_idx and topk_logit must be %zu-byte aligned", cache_align);
+  if (!aligned(workspace, 256)) return fail(KDKL_ERR_ALIGN, "workspace must be 256-byte aligned");
+  const WsLayout L = make_layout(N, 8, V, K, 0);
+  if (workspace_bytes < L.gbuf)
+    return fail(KDKL_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, L.gbuf);
+  Device dv;
+  if ((st = current_device(dv)) != KDKL_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (N == 0) {
+    const cudaError_t e = cudaMemsetAsync(workspace, 0, 256, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+    return ok();
+  }
+  if ((st = run_prepass(c, L, s)) != KDKL_OK) return st;
+  return ok();
+}
+
 const uint32_t* kdkl_n_valid_device(const void* workspace) {
   return workspace ? reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(workspace) + 4) : nullptr;
 }
@@ -882,7 +970,7 @@ const uint32_t* kdkl_n_valid_device(const void* workspace) {
 // ---------------------------------------------------------------- teacher top-K producer
 namespace {
 struct TopkLayout {
-  size_t header = 0, tv = 0, ti = 0, total = 0;
+  size_t header = 0, sync = 0, tv = 0, ti = 0, total = 0;
   int s_cap = 1;
 };
 
@@ -892,6 +980,8 @@ TopkLayout topk_layout(int64_t N, int32_t K) {
   // enough partial slots for either tile height (256-row pairs or 128-row CTAs)
   const size_t slots = static_cast<size_t>((N + 255) / 256 + 1) * 256 * L.s_cap * K;
   size_t off = 256;
+  L.sync = off;
+  off += static_cast<size_t>(kSyncSlots) * 8;
   L.tv = off;
   off = align_up(off + slots * 4, 256);
   L.ti = off;
@@ -958,15 +1048,19 @@ kdkl_status kdkl_teacher_topk(const void* hidden, const void* W, int64_t N, int3
   ep.topk_K = K;
   ep.part_tv = at<float>(workspace, L.tv);
   ep.part_ti = at<int>(workspace, L.ti);
+  ep.topk_cap = static_cast<int64_t>((L.ti - L.tv) / 4);
   ep.flags = at<uint32_t>(workspace, 0);
   ep.exp_scale = 1.4426950408889634f;
   ep.inv_tau_s = 1.0f;
   const int grid = pr.grid(sc.units);
+  if ((e = arm_sync(sc, at<unsigned long long>(workspace, L.sync), grid, true, s)) != cudaSuccess)
+    return cuda_fail(e, "cudaMemsetAsync");
   if ((e = timed(kTTopK, s, [&] { return launch_gemm(kEpiTopK, 256, true, tmA, tmB, tmA, sc, ep, grid, s); })) !=
       cudaSuccess)
     return cuda_fail(e, "top-K GEMM launch");
   if ((e = timed(kTTopKMerge, s, [&] {
-         return launch_topk_merge(ep.part_tv, ep.part_ti, splits, pr.rows, K, N, topk_idx, topk_logit, s);
+         return launch_topk_merge(ep.part_tv, ep.part_ti, splits, pr.rows, K, N, topk_idx, topk_logit, ep.topk_cap,
+                                  ep.flags, s);
        })) != cudaSuccess)
     return cuda_fail(e, "top-K merge launch");
   return ok();

@@ -24,6 +24,7 @@ inline int list_pitch(int K) { return ((K + 2) + 3) & ~3; }   // K entries + a h
 //   [2] ticket of the loss reduction
 struct WsLayout {
   size_t header = 0;       // 256 bytes
+  size_t sync = 0;         // [kSyncSlots] uint64 positions of a synchronised GEMM launch
   size_t sidx = 0;         // [N, Kp] int32 sorted unique indices (sentinel padded)
   size_t sprob = 0;        // [N, Kp] f32 teacher probabilities aligned with sidx
   size_t negent = 0;       // [N] f32 gamma * sum_v P_T log P_T of the teacher row
@@ -54,12 +55,31 @@ WsLayout make_layout(int64_t N, int32_t d, int32_t V, int32_t K, int64_t chunk_t
 //     W tiles (for launches whose row blocks all fit in L2).
 constexpr int kRowMajor = 1;
 constexpr int kSplitMajor = 2;
+//
+// Lockstep of a row-stream launch (sync_window > 0): the CTA groups that run units of
+// the same vocabulary split in the same round (round k = units [k G, k G + G) for G
+// groups; group g runs unit g + k G) stream the same W tiles, which only one DRAM
+// read serves while they stay close together.  Each group publishes its position
+// (unit + 1) << 32 | (tile - first tile of the unit) in prog[group] as it starts a
+// tile, and the even CTA's producer holds back tile r of a unit until every peer
+// group of that round and split has reached tile r - sync_window.  prog must be
+// zeroed before the launch.  A wait that lasts longer than kSyncSoftLimitNs gives
+// up and the group stops holding back for the rest of its unit; waiting never
+// changes results, only how far the groups drift apart.
+enum L2Priority { kL2Normal = 0, kL2Last = 1, kL2First = 2 };
+constexpr int kSyncSlots = 1024;                          // groups a synchronised launch may have
+constexpr unsigned long long kSyncSoftLimitNs = 1000000;  // 1 ms
 struct Sched {
   int units;
   int splits;
   int n_tiles;
   int k_blocks;
   int row_stream;
+  int sync_window;
+  unsigned long long* prog;
+  // L2 eviction priority of the A and B operand loads (kL2Normal = 0, kL2Last, kL2First)
+  int l2_a;
+  int l2_b;
 };
 
 // Parameters of the fused epilogues (the union of what each kind needs).
@@ -73,10 +93,11 @@ struct EpiParams {
   const float* sprob;
   int Kp;
   const uint8_t* rowmask;
-  // forward partials
+  // forward partials (part_cap slots per plane)
   float* part_m;
   float* part_s;
   float* part_a;
+  int64_t part_cap;
   // student temperature: exp_scale = log2(e) / tau_s, inv_tau_s = 1 / tau_s
   float exp_scale;
   float inv_tau_s;
@@ -95,6 +116,7 @@ struct EpiParams {
   int topk_K;
   float* part_tv;
   int* part_ti;
+  int64_t topk_cap;    // entries of part_tv / part_ti
 };
 
 // kEpiLseStore: the forward's online log-sum-exp and gather (as kEpiLse), and
@@ -124,17 +146,18 @@ cudaError_t launch_prepass(int cache_format, const void* topk_idx, const void* t
 cudaError_t launch_gpass(const float* z, int64_t ldz, uint16_t* G, int64_t ldg, int64_t nc, int V,
                          int64_t row_offset, const int* sidx, const float* sprob, int Kp, const uint8_t* rowmask,
                          const float* wsum, const float* lse, const uint32_t* n_valid, const float* grad_loss,
-                         float student_tau, cudaStream_t stream);
+                         float student_tau, uint32_t* flags, cudaStream_t stream);
 
 // launch_merge: rows [0, N) of the pointers given (a chunk passes offset per-row
 // pointers); their 256-row block sums land at blocksum[block_base + b], and the
 // launch that completes block total_blocks - 1 of the step (0 = this launch's
-// grid) sums all total_blocks in order into *loss.
+// grid) sums all total_blocks in order into *loss.  part_cap = slots per partial
+// plane (checked in the bounds-checking build).
 cudaError_t launch_merge(const float* part_m, const float* part_s, const float* part_a, int splits,
                          int rows_per_block, float student_tau, const float* negent, const float* wsum,
                          const uint8_t* rowmask, int64_t N, float* lse, float* loss, double* blocksum,
                          uint32_t* header, const uint32_t* n_valid, int64_t block_base, int64_t total_blocks,
-                         cudaStream_t stream);
+                         int64_t part_cap, cudaStream_t stream);
 
 // GEMM kinds: A/B majorness and epilogue are fixed per kind.
 //   kEpiLse      : A = hidden K-major, B = W K-major, BN = 256, row-stream
@@ -151,7 +174,8 @@ cudaError_t launch_gemm(int kind, int BN, bool pair, const CUtensorMap& tmA, con
 // Merges the per-split heaps of the top-K producer into each row's K entries,
 // ordered by (logit descending, index ascending).
 cudaError_t launch_topk_merge(const float* part_tv, const int* part_ti, int splits, int rows_per_block, int K,
-                              int64_t N, int32_t* topk_idx, float* topk_logit, cudaStream_t stream);
+                              int64_t N, int32_t* topk_idx, float* topk_logit, int64_t part_cap, uint32_t* flags,
+                              cudaStream_t stream);
 
 // Bounded-wait self-test (see kdkl_selftest_wait_timeout).
 cudaError_t launch_wait_selftest(uint32_t* flags, uint64_t limit_ns, uint64_t* waited_ns, cudaStream_t stream);

@@ -19,6 +19,7 @@
 // into the loss, chunks are discarded, the backward recomputes them; llm-wiki
 // note, section "Fused Chunked KL": softmax, log and KL fused in one kernel).
 #include <cfloat>
+#include <climits>
 #include <cmath>
 
 #include <atomic>
@@ -150,8 +151,10 @@ __global__ void __launch_bounds__(kPreWarps * 32)
           const int other = key[j];
           rank += (other < mine) || (other == mine && j < k);
         }
-        skey[rank] = mine;
-        sp[rank] = pv[k];
+        if (dbg_ok(rank < K, header)) {
+          skey[rank] = mine;
+          sp[rank] = pv[k];
+        }
       }
     }
     __syncwarp();
@@ -177,7 +180,7 @@ __global__ void __launch_bounds__(kPreWarps * 32)
       }
       const uint32_t ballot = __ballot_sync(0xffffffffu, start);
       const int pos = cnt + __popc(ballot & ((1u << lane) - 1u));
-      if (start) {
+      if (start && dbg_ok(pos < Kp - 1, header)) {   // room for the sentinel after the list
         key[pos] = kk;
         pv[pos] = gamma * pm;
         if (pm > 0.f) ent += pm * logf(pm);
@@ -201,7 +204,7 @@ __global__ void __launch_bounds__(kPreWarps * 32)
           }
           if (lo < cnt && key[lo] == lab) {
             pv[lo] += beta;
-          } else {
+          } else if (dbg_ok(cnt + 1 < Kp, header)) {
             for (int t = cnt; t > lo; --t) {
               key[t] = key[t - 1];
               pv[t] = pv[t - 1];
@@ -268,13 +271,14 @@ __global__ void __launch_bounds__(kMergeThreads)
                  const float* __restrict__ negent, const float* __restrict__ wsum,
                  const uint8_t* __restrict__ rowmask, int64_t N, float* __restrict__ lse,
                  float* __restrict__ loss, double* __restrict__ blocksum, uint32_t* __restrict__ header,
-                 const uint32_t* __restrict__ n_valid, int64_t block_base, int64_t total_blocks) {
+                 const uint32_t* __restrict__ n_valid, int64_t block_base, int64_t total_blocks,
+                 int64_t part_cap) {
   __shared__ double s_red[kMergeThreads / 32];
   __shared__ bool s_last;
   const int64_t n = static_cast<int64_t>(blockIdx.x) * kMergeThreads + threadIdx.x;
   double kl = 0.0;
-  if (n < N) {
-    const int64_t rb = n / rows_per_block;
+  const int64_t rb = n / rows_per_block;
+  if (n < N && dbg_ok((rb * splits + splits) * rows_per_block <= part_cap, header)) {
     const int r = static_cast<int>(n - rb * rows_per_block);
     float M = -INFINITY;
     for (int j = 0; j < splits; ++j) M = fmaxf(M, part_m[(rb * splits + j) * rows_per_block + r]);
@@ -320,12 +324,12 @@ cudaError_t launch_merge(const float* part_m, const float* part_s, const float* 
                          int rows_per_block, float student_tau, const float* negent, const float* wsum,
                          const uint8_t* rowmask, int64_t N, float* lse, float* loss, double* blocksum,
                          uint32_t* header, const uint32_t* n_valid, int64_t block_base, int64_t total_blocks,
-                         cudaStream_t stream) {
+                         int64_t part_cap, cudaStream_t stream) {
   const int grid = static_cast<int>((N + kMergeThreads - 1) / kMergeThreads);
   if (total_blocks <= 0) total_blocks = grid;
   merge_kernel<<<grid, kMergeThreads, 0, stream>>>(part_m, part_s, part_a, splits, rows_per_block,
                                                    1.0f / student_tau, negent, wsum, rowmask, N, lse, loss,
-                                                   blocksum, header, n_valid, block_base, total_blocks);
+                                                   blocksum, header, n_valid, block_base, total_blocks, part_cap);
   return cudaGetLastError();
 }
 
@@ -357,11 +361,12 @@ struct GemmCfg {
   static constexpr int kTxBytes = (PAIR ? 2 : 1) * kStageBytes;       // counted on the MMA's barrier
   // per-epilogue-warp staging: grad 2 x 2 KB (32 x 32 bf16), dW 4 KB (32 x 32 fp32),
   // stored logits 2 x 4 KB (32 x 32 fp32); top-K: the heaps of all 128 rows
-  static constexpr int kEpiWarpBytes = (KIND == kEpiLseStore) ? 8192 : 4096;
+  // dW: 2 x 4 KB (32 x 32 fp32, the old block loaded and the new one stored through it)
+  static constexpr int kEpiWarpBytes = (KIND == kEpiLseStore || KIND == kEpiRmwF32) ? 8192 : 4096;
   static constexpr int kEpiBytes = (KIND == kEpiGrad || KIND == kEpiRmwF32 || KIND == kEpiLseStore)
                                        ? 4 * kEpiWarpBytes
                                        : (KIND == kEpiTopK ? kTopKMax * kBM * 6 : 0);
-  static constexpr int kBarBytes = 256;
+  static constexpr int kBarBytes = 512;
   static constexpr int kSmemLimit = 232448;
   static constexpr int kStagesFit = (kSmemLimit - 1024 - kEpiBytes - kBarBytes) / kStageBytes;
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
@@ -400,6 +405,56 @@ __device__ __forceinline__ void unit_range(const Sched& sc, int u, int& mb, int&
     t0 = u - mb * sc.n_tiles;
     t1 = t0 + 1;
   }
+}
+
+// Position word a group publishes as it starts relative tile r of unit u.
+__device__ __forceinline__ unsigned long long sync_word(int u, int r) {
+  return (static_cast<unsigned long long>(u + 1) << 32) | static_cast<unsigned int>(r);
+}
+
+// Whole warp (the producer warp of an even CTA): the smallest relative tile that the
+// other groups running a unit of split j in unit u's round have reached in that unit
+// (a peer already past that unit counts as INT_MAX, one not yet in it as -1), waiting
+// until it is at least r_need.  Returns -2 if the wait gave up (kSyncSoftLimitNs).
+__device__ int wait_split_peers(const Sched& sc, int u, int group, int ngroups, int j, int r_need, int lane,
+                                uint32_t* flags) {
+  const int round0 = u - group;                  // group g runs units g + k G: this round is [k G, k G + G)
+  const int round1 = min(round0 + ngroups, sc.units);
+  int first, last, step;
+  if (sc.row_stream == kSplitMajor) {            // units of split j are j rb ... j rb + rb - 1
+    const int rb = sc.units / sc.splits;
+    first = max(round0, j * rb);
+    last = min(round1, (j + 1) * rb);
+    step = 1;
+  } else {                                       // units of split j are those with u % splits == j
+    first = round0 + ((j - round0 % sc.splits) % sc.splits + sc.splits) % sc.splits;
+    last = round1;
+    step = sc.splits;
+  }
+  const uint64_t t0 = globaltimer_ns();
+  int seen = INT_MAX;
+  for (int base = first; base < last; base += 32 * step) {
+    const int up = base + lane * step;
+    const bool mine = up < last && up != u;
+    const volatile unsigned long long* slot =
+        sc.prog + ((mine && dbg_ok(up - round0 < ngroups && ngroups <= kSyncSlots, flags)) ? up - round0 : 0);
+    int rel = INT_MAX;
+    while (true) {
+      if (mine) {
+        const unsigned long long w = *slot;
+        const unsigned long long hi = w >> 32, want = static_cast<unsigned long long>(up + 1);
+        rel = hi > want ? INT_MAX : (hi == want ? static_cast<int>(w & 0xFFFFFFFFull) : -1);
+      }
+      const int lo = __reduce_min_sync(0xffffffffu, rel);
+      if (lo >= r_need) {
+        seen = min(seen, lo);
+        break;
+      }
+      if (__any_sync(0xffffffffu, globaltimer_ns() - t0 > kSyncSoftLimitNs)) return -2;
+      __nanosleep(128);
+    }
+  }
+  return seen;
 }
 
 // z[off] for a run-time off in [0, 32) without dynamic register indexing.
@@ -445,7 +500,8 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* acc_full = bars + 2 * C::kStages;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* ebar = drain + 1;             // dW epilogue: one load barrier per staging buffer (4 warps x 2)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ebar + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -463,13 +519,14 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&acc_empty[b], C::kAccEmptyArrivals);
     }
     mbar_init(drain, 1);
+    for (int b = 0; b < 8; ++b) mbar_init(&ebar[b], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
-    if (KIND == kEpiGrad || KIND == kEpiLseStore) tma_prefetch_desc(&tmOut);
+    if (KIND == kEpiGrad || KIND == kEpiLseStore || KIND == kEpiRmwF32) tma_prefetch_desc(&tmOut);
   }
   if (warp == 1) {
     if (PAIR) {
@@ -489,35 +546,73 @@ __global__ void __launch_bounds__(192, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      for (int u = group; u < sc.units; u += ngroups) {
-        int mb, uj, t0, t1;
-        unit_range(sc, u, mb, uj, t0, t1);
-        const int arow = mb * C::kMmaM + static_cast<int>(rank) * kBM;   // this CTA's A rows
-        for (int t = t0; t < t1; ++t) {
-          const int bcol = t * BN + static_cast<int>(rank) * C::kCtaN;  // this CTA's B rows (N)
+    // Lane 0 issues the copies; the whole warp takes part in the lockstep wait.
+    int stage = 0;
+    uint32_t phase = 0;
+    bool wrapped = false;    // every stage has been filled at least once
+    bool stop = false;
+    const bool sync_on = sc.sync_window > 0 && sc.row_stream != 0 && rank == 0;
+    const bool hints = (sc.l2_a | sc.l2_b) != 0;
+    const uint64_t pol_a = l2_policy(sc.l2_a), pol_b = l2_policy(sc.l2_b);
+    for (int u = group; u < sc.units && !stop; u += ngroups) {
+      int mb, uj, t0, t1;
+      unit_range(sc, u, mb, uj, t0, t1);
+      const int arow = mb * C::kMmaM + static_cast<int>(rank) * kBM;   // this CTA's A rows
+      bool hold = sync_on;
+      int seen = -1;          // every peer had reached this relative tile at the last look
+      for (int t = t0; t < t1 && !stop; ++t) {
+        if (sync_on) {
+          const int need = t - t0 - sc.sync_window;
+          if (hold && need > seen) {
+            const int got = wait_split_peers(sc, u, group, ngroups, uj, need, lane, ep.flags);
+            if (got == -2) hold = false;
+            else seen = got;
+          }
+          if (lane == 0) *reinterpret_cast<volatile unsigned long long*>(sc.prog + group) = sync_word(u, t - t0);
+        }
+        int lstop = 0;
+        if (lane == 0) {
+          int bcol = t * BN + static_cast<int>(rank) * C::kCtaN;  // this CTA's B rows (N)
+          if (C::kBmn && !dbg_ok((bcol & 7) == 0, ep.flags)) bcol &= ~7;   // x of an MN-major bf16 box
           for (int kb = 0; kb < sc.k_blocks; ++kb) {
-            if (!mbar_wait(&empty[stage], phase ^ 1u, ab)) goto producer_done;
+            if (!mbar_wait(&empty[stage], phase ^ 1u, ab)) {
+              lstop = 1;
+              break;
+            }
             uint8_t* a = sA + stage * C::kABytes;
             uint8_t* b = sB + stage * C::kBBytes;
             if (PAIR) {
               // both CTAs' bytes are counted on the even CTA's barrier
               const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
               if (rank == 0) mbar_arrive_expect_tx(&full[stage], C::kTxBytes);
-              if (C::kAmn) {
-                tma_load_2d_pair(a, &tmA, bar0, arow, kb * kBK);
-                tma_load_2d_pair(a + 8192, &tmA, bar0, arow + 64, kb * kBK);
-              } else {
-                tma_load_2d_pair(a, &tmA, bar0, kb * kBK, arow);
-              }
-              if (C::kBmn) {
+              if (hints) {
+                if (C::kAmn) {
+                  tma_load_2d_pair_hint(a, &tmA, bar0, arow, kb * kBK, pol_a);
+                  tma_load_2d_pair_hint(a + 8192, &tmA, bar0, arow + 64, kb * kBK, pol_a);
+                } else {
+                  tma_load_2d_pair_hint(a, &tmA, bar0, kb * kBK, arow, pol_a);
+                }
+                if (C::kBmn) {
 #pragma unroll
-                for (int q = 0; q < C::kBAtoms; ++q)
-                  tma_load_2d_pair(b + q * 8192, &tmB, bar0, bcol + q * 64, kb * kBK);
+                  for (int q = 0; q < C::kBAtoms; ++q)
+                    tma_load_2d_pair_hint(b + q * 8192, &tmB, bar0, bcol + q * 64, kb * kBK, pol_b);
+                } else {
+                  tma_load_2d_pair_hint(b, &tmB, bar0, kb * kBK, bcol, pol_b);
+                }
               } else {
-                tma_load_2d_pair(b, &tmB, bar0, kb * kBK, bcol);
+                if (C::kAmn) {
+                  tma_load_2d_pair(a, &tmA, bar0, arow, kb * kBK);
+                  tma_load_2d_pair(a + 8192, &tmA, bar0, arow + 64, kb * kBK);
+                } else {
+                  tma_load_2d_pair(a, &tmA, bar0, kb * kBK, arow);
+                }
+                if (C::kBmn) {
+#pragma unroll
+                  for (int q = 0; q < C::kBAtoms; ++q)
+                    tma_load_2d_pair(b + q * 8192, &tmB, bar0, bcol + q * 64, kb * kBK);
+                } else {
+                  tma_load_2d_pair(b, &tmB, bar0, kb * kBK, bcol);
+                }
               }
             } else {
               mbar_arrive_expect_tx(&full[stage], C::kTxBytes);
@@ -538,11 +633,25 @@ __global__ void __launch_bounds__(192, 1)
             if (++stage == C::kStages) {
               stage = 0;
               phase ^= 1u;
+              wrapped = true;
             }
           }
         }
+        stop = __shfl_sync(0xffffffffu, lstop, 0) != 0;
       }
-    producer_done:;
+    }
+    if (lane == 0 && rank == 0 && *abort_flag) {
+      // The kernel is giving up: before shared memory is released, wait (bounded) until
+      // the copies already issued have landed.  The even CTA's full barriers count
+      // both CTAs' bytes, so the last issued phase of each stage covers the pair.
+      const uint64_t w0 = globaltimer_ns();
+      for (int s2 = 0; s2 < C::kStages; ++s2) {
+        if (!wrapped && s2 >= stage) break;              // never filled
+        const uint32_t par = s2 < stage ? phase : (phase ^ 1u);
+        const uint32_t a = smem_u32(&full[s2]);
+        while (!mbar_try_wait(a, par) && globaltimer_ns() - w0 < kDrainLimitNs) {
+        }
+      }
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -621,6 +730,9 @@ __global__ void __launch_bounds__(192, 1)
     uint8_t* wbuf = sEpi + (warp - 2) * C::kEpiWarpBytes;   // this warp's staging
     uint8_t* wbuf_all = sEpi;                    // top-K heaps of all 128 rows
     int sbuf = 0;
+    // dW: staging buffer of the next TMA chunk, load-barrier phase bits and loads in flight
+    uint64_t* wbar = ebar + 2 * (warp - 2);
+    uint32_t dw_phase = 0, dw_pending = 0;
     for (int u = group; u < sc.units; u += ngroups) {
       int mb, uj, t0, t1;
       unit_range(sc, u, mb, uj, t0, t1);
@@ -667,6 +779,7 @@ __global__ void __launch_bounds__(192, 1)
           lst = ep.sidx + grow * ep.Kp;
           lsp = ep.sprob + grow * ep.Kp;
           kpos = lower_bound_list(lst, ep.Kp, t0 * BN);
+          if (!dbg_ok(kpos < ep.Kp, ep.flags)) kpos = ep.Kp - 1;
           nxt = lst[kpos];
           nxtp = lsp[kpos];
         }
@@ -678,10 +791,32 @@ __global__ void __launch_bounds__(192, 1)
         // columns of this tile: [t * BN, col_lim); a last 32-column chunk that runs past
         // BN reads unused TMEM columns, which the stores below skip
         const int col_lim = min(ep.Ncols, t * BN + BN);
+        // dW: a 32-column chunk that lies inside the tile goes through TMA (columns past d
+        // and rows past V are clipped by the tensor map); with BN = 240 the last chunk holds
+        // 16 columns and takes the per-thread path.  When accumulating, the old block of
+        // chunk c + 1 is loaded while chunk c is processed.
+        auto dw_tma_chunk = [&](int cc) {
+          const int cl = t * BN + cc * 32;
+          return cl < col_lim && cl + 32 <= t * BN + BN;
+        };
+        auto dw_load = [&](int cc, int b) {
+          if (lane == 0) {
+            bulk_wait_read<0>();   // the last store out of buffer b has read it
+            mbar_arrive_expect_tx(&wbar[b], 4096);
+            const int lx = t * BN + cc * 32;
+            tma_load_2d(wbuf + b * 4096, &tmOut, &wbar[b], dbg_ok((lx & 3) == 0, ep.flags) ? lx : (lx & ~3),
+                        row0 + q * 32);
+          }
+          dw_pending |= 1u << b;
+          __syncwarp();
+        };
+        if (KIND == kEpiRmwF32 && ep.accumulate && dw_tma_chunk(0)) dw_load(0, sbuf);
 #pragma unroll 1
         for (int c = 0; c < (BN + 31) / 32; ++c) {
           const int col = t * BN + c * 32;
           if (col >= col_lim) break;
+          if (KIND == kEpiRmwF32 && ep.accumulate && dw_tma_chunk(c) && dw_tma_chunk(c + 1))
+            dw_load(c + 1, sbuf ^ 1);
           float v[32];
           tmem_ld32(tbase + c * 32, v);
           tmem_wait_ld();
@@ -702,7 +837,7 @@ __global__ void __launch_bounds__(192, 1)
                              __float_as_uint(v[c16 * 4 + 3]));
               fence_proxy_async_smem();
               __syncwarp();
-              if (lane == 0) {
+              if (lane == 0 && dbg_ok((col & 3) == 0 && col >= 0 && row0 + q * 32 >= 0, ep.flags)) {
                 tma_store_2d(&tmOut, buf, col, row0 + q * 32);
                 bulk_commit();
               }
@@ -724,6 +859,10 @@ __global__ void __launch_bounds__(192, 1)
             s_run = s_run * ex2_approx((m_run - mn) * es) + acc_s;
             m_run = mn;
             while (nxt < col + 32) {
+              if (!dbg_ok(nxt >= col && kpos + 1 < ep.Kp, ep.flags)) {
+                nxt = kSentinel;
+                break;
+              }
               a_run = fmaf(nxtp, pick32(v, static_cast<uint32_t>(nxt - col)), a_run);
               ++kpos;
               nxt = lst[kpos];
@@ -734,6 +873,10 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) g[j] = cnw * ex2_approx(fmaf(v[j], es, -lse_l2));
             while (nxt < col + 32) {
+              if (!dbg_ok(nxt >= col && kpos + 1 < ep.Kp, ep.flags)) {
+                nxt = kSentinel;
+                break;
+              }
               const uint32_t off = static_cast<uint32_t>(nxt - col);
               const float cp = cn * nxtp;
 #pragma unroll
@@ -755,7 +898,7 @@ __global__ void __launch_bounds__(192, 1)
                            pack_bf16x2(g[c16 * 8 + 4], g[c16 * 8 + 5]), pack_bf16x2(g[c16 * 8 + 6], g[c16 * 8 + 7]));
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) {
+            if (lane == 0 && dbg_ok((col & 7) == 0 && col >= 0 && row0 + q * 32 >= 0, ep.flags)) {
               tma_store_2d(&tmOut, buf, col, row0 + q * 32);
               bulk_commit();
             }
@@ -818,36 +961,48 @@ __global__ void __launch_bounds__(192, 1)
               }
             }
           } else {  // kEpiRmwF32
-            // Transpose the warp's 32 x 32 fp32 block through shared memory so
-            // that each global access is one full 128-byte row segment.
-            // 16-byte chunk q of row r sits at chunk (q ^ (r & 7)): conflict-free both ways.
-            const uint32_t fb = smem_u32(wbuf);
-#pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4)
-              st_shared_v4(fb + static_cast<uint32_t>(lane * 128 + ((q4 ^ (lane & 7)) << 4)),
-                           __float_as_uint(v[q4 * 4 + 0]), __float_as_uint(v[q4 * 4 + 1]),
-                           __float_as_uint(v[q4 * 4 + 2]), __float_as_uint(v[q4 * 4 + 3]));
-            __syncwarp();
             const int wrow0 = row0 + q * 32;
-            const bool cv = (col + lane) < col_lim;
-            float r[32];
+            if (dw_tma_chunk(c)) {
+              // the warp's 32 rows x 32 fp32 columns in the 128-byte-swizzled layout of the
+              // tensor map (16-byte chunk c16 of row r at c16 ^ (r & 7)): thread = row
+              uint8_t* buf = wbuf + sbuf * 4096;
+              const uint32_t sw = static_cast<uint32_t>(lane & 7);
+              const uint32_t row_addr = smem_u32(buf) + static_cast<uint32_t>(lane) * 128u;
+              if (ep.accumulate) {
+                if (!mbar_wait(&wbar[sbuf], (dw_phase >> sbuf) & 1u, ab)) goto epi_done;
+                dw_phase ^= 1u << sbuf;
+                dw_pending &= ~(1u << sbuf);
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              r[i] = ld_shared_f32(fb + static_cast<uint32_t>(i * 128 + (((lane >> 2) ^ (i & 7)) << 4) +
-                                                              (lane & 3) * 4));
-            __syncwarp();
-            float* base = ep.dW + static_cast<int64_t>(wrow0) * ep.ldo + col + lane;
-            if (ep.accumulate) {
-              float old[32];
+                for (int c16 = 0; c16 < 8; ++c16) {
+                  const float4 o = ld_shared_v4f(row_addr + ((static_cast<uint32_t>(c16) ^ sw) << 4));
+                  v[c16 * 4 + 0] += o.x;
+                  v[c16 * 4 + 1] += o.y;
+                  v[c16 * 4 + 2] += o.z;
+                  v[c16 * 4 + 3] += o.w;
+                }
+              } else {
+                if (lane == 0) bulk_wait_read<1>();   // the store before last out of this buffer has read it
+                __syncwarp();
+              }
 #pragma unroll
-              for (int i = 0; i < 32; ++i)
-                old[i] = (cv && wrow0 + i < ep.M) ? base[static_cast<int64_t>(i) * ep.ldo] : 0.f;
+              for (int c16 = 0; c16 < 8; ++c16)
+                st_shared_v4(row_addr + ((static_cast<uint32_t>(c16) ^ sw) << 4), __float_as_uint(v[c16 * 4 + 0]),
+                             __float_as_uint(v[c16 * 4 + 1]), __float_as_uint(v[c16 * 4 + 2]),
+                             __float_as_uint(v[c16 * 4 + 3]));
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0 && dbg_ok((col & 3) == 0 && col >= 0 && wrow0 >= 0, ep.flags)) {
+                tma_store_2d(&tmOut, buf, col, wrow0);
+                bulk_commit();
+              }
+              sbuf ^= 1;
+            } else if (rv) {
+              // a chunk cut by the tile edge: this thread's own row, element by element
+              float* dst = ep.dW + static_cast<int64_t>(row) * ep.ldo;
 #pragma unroll
-              for (int i = 0; i < 32; ++i) r[i] += old[i];
+              for (int j = 0; j < 32; ++j)
+                if (col + j < col_lim) dst[col + j] = (ep.accumulate ? dst[col + j] : 0.f) + v[j];
             }
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (cv && wrow0 + i < ep.M) base[static_cast<int64_t>(i) * ep.ldo] = r[i];
           }
         }
         tc_fence_before();
@@ -862,7 +1017,8 @@ __global__ void __launch_bounds__(192, 1)
       if (KIND == kEpiTopK && rv) {
         const int64_t slot = (uslot * C::kMmaM + static_cast<int>(rank) * kBM + row_local) *
                              ep.topk_K;
-        for (int k = 0; k < ep.topk_K; ++k) {
+        const int kw = dbg_ok(slot + ep.topk_K <= ep.topk_cap, ep.flags) ? ep.topk_K : 0;
+        for (int k = 0; k < kw; ++k) {
           const int rel = hi[k * kBM];
           ep.part_tv[slot + k] = hv[k * kBM];
           ep.part_ti[slot + k] = rel == kTopKEmpty ? kSentinel : ubase + rel;
@@ -870,13 +1026,23 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (kLseLike && rv) {
         const int64_t slot = uslot * C::kMmaM + static_cast<int>(rank) * kBM + row_local;
-        ep.part_m[slot] = m_run;
-        ep.part_s[slot] = s_run;
-        ep.part_a[slot] = a_run;
+        if (dbg_ok(slot < ep.part_cap, ep.flags)) {
+          ep.part_m[slot] = m_run;
+          ep.part_s[slot] = s_run;
+          ep.part_a[slot] = a_run;
+        }
       }
     }
   epi_done:
-    if (KIND == kEpiGrad || KIND == kEpiLseStore) {
+    if (KIND == kEpiRmwF32 && lane == 0 && dw_pending) {
+      // a load of an old dW block may still be landing (abort path): bounded wait
+      const uint64_t w0 = globaltimer_ns();
+      for (int b2 = 0; b2 < 2; ++b2)
+        if (dw_pending & (1u << b2))
+          while (!mbar_try_wait(smem_u32(&wbar[b2]), (dw_phase >> b2) & 1u) && globaltimer_ns() - w0 < kDrainLimitNs) {
+          }
+    }
+    if (KIND == kEpiGrad || KIND == kEpiLseStore || KIND == kEpiRmwF32) {
       if (lane == 0) bulk_wait<0>();
       __syncwarp();
     }
@@ -1030,7 +1196,7 @@ __global__ void __launch_bounds__(kGPassThreads)
                  int64_t row_offset, const int* __restrict__ sidx, const float* __restrict__ sprob, int Kp,
                  const uint8_t* __restrict__ rowmask, const float* __restrict__ wsum,
                  const float* __restrict__ lse, const uint32_t* __restrict__ n_valid,
-                 const float* __restrict__ grad_loss, float inv_tau_s, float exp_scale) {
+                 const float* __restrict__ grad_loss, float inv_tau_s, float exp_scale, uint32_t* __restrict__ flags) {
   const int64_t n = blockIdx.x;
   const int64_t grow = row_offset + n;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1087,8 +1253,8 @@ __global__ void __launch_bounds__(kGPassThreads)
       float gv[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) gv[j] = cnw * ex2_approx(fmaf(v[u][j], es, -lse_l2));
-      while (lst[kpos] < g0) ++kpos;
-      for (int k = kpos; lst[k] < g0 + 128; ++k) {
+      while (lst[kpos] < g0 && dbg_ok(kpos + 1 < Kp, flags)) ++kpos;
+      for (int k = kpos; lst[k] < g0 + 128 && dbg_ok(k + 1 < Kp, flags); ++k) {
         const uint32_t off = static_cast<uint32_t>(lst[k] - c0);
         const float cp = cn * lsp[k];
 #pragma unroll
@@ -1109,11 +1275,11 @@ __global__ void __launch_bounds__(kGPassThreads)
 cudaError_t launch_gpass(const float* z, int64_t ldz, uint16_t* G, int64_t ldg, int64_t nc, int V,
                          int64_t row_offset, const int* sidx, const float* sprob, int Kp, const uint8_t* rowmask,
                          const float* wsum, const float* lse, const uint32_t* n_valid, const float* grad_loss,
-                         float student_tau, cudaStream_t stream) {
+                         float student_tau, uint32_t* flags, cudaStream_t stream) {
   if (nc <= 0) return cudaSuccess;
   gpass_kernel<<<static_cast<unsigned>(nc), kGPassThreads, 0, stream>>>(
       z, ldz, G, ldg, V, row_offset, sidx, sprob, Kp, rowmask, wsum, lse, n_valid, grad_loss, 1.0f / student_tau,
-      1.4426950408889634f / student_tau);
+      1.4426950408889634f / student_tau, flags);
   return cudaGetLastError();
 }
 
@@ -1154,7 +1320,7 @@ __device__ __forceinline__ int topk_key_index(uint64_t key) {
 __global__ void __launch_bounds__(kTopKMergeWarps * 32)
     topk_merge_kernel(const float* __restrict__ part_tv, const int* __restrict__ part_ti, int splits,
                       int rows_per_block, int K, int64_t N, int32_t* __restrict__ topk_idx,
-                      float* __restrict__ topk_logit) {
+                      float* __restrict__ topk_logit, int64_t part_cap, uint32_t* __restrict__ flags) {
   constexpr int kPerLane = kMergeCand / 32;
   __shared__ uint32_t s_hist[kTopKMergeWarps][256];
   __shared__ uint64_t s_sel[kTopKMergeWarps][kTopKMax];
@@ -1178,7 +1344,7 @@ __global__ void __launch_bounds__(kTopKMergeWarps * 32)
       if (c < C) {
         const int j = c / K, k = c - j * K;
         const int64_t slot = ((rb * splits + j) * rows_per_block + r) * K + k;
-        key[i] = topk_key(part_tv[slot], part_ti[slot]);
+        if (dbg_ok(slot < part_cap, flags)) key[i] = topk_key(part_tv[slot], part_ti[slot]);
       }
     }
     // radix select: after pass p, `prefix` holds the top p+1 bytes of the K-th
@@ -1239,7 +1405,8 @@ __global__ void __launch_bounds__(kTopKMergeWarps * 32)
     for (int i = 0; i < kPerLane; ++i) {
       const bool take = key[i] > kth;
       const uint32_t b = __ballot_sync(0xffffffffu, take);
-      if (take) sel[base + __popc(b & ((1u << lane) - 1u))] = key[i];
+      if (take && dbg_ok(base + __popc(b & ((1u << lane) - 1u)) < kTopKMax, flags))
+        sel[base + __popc(b & ((1u << lane) - 1u))] = key[i];
       base += __popc(b);
     }
     for (int k = base + lane; k < K; k += 32) sel[k] = kth;
@@ -1272,12 +1439,13 @@ __global__ void __launch_bounds__(kTopKMergeWarps * 32)
 }
 
 cudaError_t launch_topk_merge(const float* part_tv, const int* part_ti, int splits, int rows_per_block, int K,
-                              int64_t N, int32_t* topk_idx, float* topk_logit, cudaStream_t stream) {
+                              int64_t N, int32_t* topk_idx, float* topk_logit, int64_t part_cap, uint32_t* flags,
+                              cudaStream_t stream) {
   if (splits * K > kMergeCand) return cudaErrorInvalidValue;
   const int64_t blocks = (N + kTopKMergeWarps - 1) / kTopKMergeWarps;
   const int grid = static_cast<int>(blocks < 4096 ? blocks : 4096);
   topk_merge_kernel<<<grid, kTopKMergeWarps * 32, 0, stream>>>(part_tv, part_ti, splits, rows_per_block, K, N,
-                                                                topk_idx, topk_logit);
+                                                                topk_idx, topk_logit, part_cap, flags);
   return cudaGetLastError();
 }
 

@@ -19,8 +19,27 @@ constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
+// The array's address is looked up once per device and primary context: a new
+// context (after cudaDeviceReset, say) loads the module again, so the array may
+// move, and the lookup is then redone.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
 std::mutex g_mu;
 void* g_scratch_addr[kMaxDevices] = {nullptr};
+CUcontext g_scratch_ctx[kMaxDevices] = {nullptr};
 
 kdkl_status reject(kdkl_status st, const char* msg) {
   kdkl::set_last_error(msg);
@@ -48,12 +67,17 @@ extern "C" kdkl_status kdkl_forward_noalloc(const void* hidden, const void* W, c
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return reject(KDKL_ERR_UNSUPPORTED, "kdkl_forward_noalloc: no CUDA device");
   if (dev < 0 || dev >= kMaxDevices) return reject(KDKL_ERR_UNSUPPORTED, "kdkl_forward_noalloc: device index too large");
+  // The current context, if this thread has one yet (a thread whose only CUDA call so
+  // far is cudaGetDevice may not): without one the lookup below runs, which binds it.
+  CUcontext ctx = nullptr;
+  CtxGetCurrentFn get_ctx = ctx_get_current();
+  if (get_ctx && get_ctx(&ctx) != CUDA_SUCCESS) ctx = nullptr;
   void* scratch = nullptr;
   {
-    // Set-up, once per device, with that device current: the host-side name of
-    // the array is not a device address, so ask the runtime for this device's copy.
+    // Set-up, once per device and context, with that device current: the host-side
+    // name of the array is not a device address, so ask the runtime for this device's copy.
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_scratch_addr[dev]) {
+    if (!g_scratch_addr[dev] || !ctx || g_scratch_ctx[dev] != ctx) {
       void* p = nullptr;
       const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
       if (e != cudaSuccess || p == nullptr) {
@@ -61,7 +85,9 @@ extern "C" kdkl_status kdkl_forward_noalloc(const void* hidden, const void* W, c
         snprintf(msg, sizeof(msg), "kdkl_forward_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
         return reject(KDKL_ERR_CUDA, msg);
       }
+      if (get_ctx && get_ctx(&ctx) != CUDA_SUCCESS) ctx = nullptr;
       g_scratch_addr[dev] = p;
+      g_scratch_ctx[dev] = ctx;
     }
     scratch = g_scratch_addr[dev];
   }

@@ -13,7 +13,23 @@ namespace kdkl {
 // (a whole kernel runs well under this); past it the kernel records
 // KDKL_DEV_TIMEOUT, stops its loops and returns.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Budget of the bounded drains on the abort path (copies and MMAs already issued).
+constexpr uint64_t kDrainLimitNs = 100000000ull;
 constexpr uint32_t kFlagTimeout = 8u;
+constexpr uint32_t kFlagBounds = 16u;
+
+// Index checks of the bounds-checking build (compiled with -DKDKL_DEBUG): a failed
+// check sets KDKL_DEV_BOUNDS in the device flag word, and the caller skips (or
+// clamps) the access instead of making it.  In the normal build every check is the
+// constant true and compiles away.
+#ifdef KDKL_DEBUG
+__device__ __forceinline__ bool dbg_ok(bool cond, uint32_t* flags) {
+  if (!cond && flags) atomicOr(flags, kFlagBounds);
+  return cond;
+}
+#else
+__device__ __forceinline__ bool dbg_ok(bool, uint32_t*) { return true; }
+#endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -96,6 +112,26 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, uin
       : "memory");
 }
 
+// The same with an L2 eviction-priority policy (from l2_policy) for the loaded lines.
+__device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* m, uint64_t* bar, int32_t x,
+                                                 int32_t y, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+
+// L2 eviction-priority policy for the loads (createpolicy, applied to every line);
+// priority is an L2Priority.
+__device__ __forceinline__ uint64_t l2_policy(int priority) {
+  uint64_t p;
+  if (priority == kL2Last) asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  else if (priority == kL2First) asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  else asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
 // 2-D tiled store shared -> global (elements outside the map's extent are skipped).
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* src, int32_t x, int32_t y) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
@@ -119,6 +155,13 @@ __device__ __forceinline__ void bulk_wait() {
 // One 16-byte shared-memory store (kept as a single 128-bit access).
 __device__ __forceinline__ void st_shared_v4(uint32_t saddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+__device__ __forceinline__ float4 ld_shared_v4f(uint32_t saddr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(saddr)
+               : "memory");
+  return v;
 }
 
 __device__ __forceinline__ float ld_shared_f32(uint32_t saddr) {
@@ -242,6 +285,15 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
       "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
           smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d_pair_hint(void* dst, const CUtensorMap* m, uint32_t bar_cluster,
+                                                      int32_t x, int32_t y, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(x), "r"(y), "l"(policy)
       : "memory");
 }
 

@@ -176,3 +176,20 @@ def test_forward_backward_argument_checks(lib):
     assert fb(dW=0xA0004) == 3
     assert fb(chunk=-1) == 2
     assert fb(ws_bytes=need - 1) == 5 and "workspace" in K.kdkl_last_error()
+
+
+def test_count_valid_argument_checks(lib):
+    N, V, Kc = 256, 4096, 16
+    need = K.kdkl_workspace_bytes(N, 8, V, Kc)
+
+    def cv(**kw):
+        a = dict(idx=0x30000, logit=0x40000, mask=0x50000, N=N, V=V, K=Kc, tau=1.0, ws=0x80000, ws_bytes=need)
+        a.update(kw)
+        return lib.kdkl_count_valid(a["idx"], a["logit"], a["mask"], a["N"], a["V"], a["K"], a["tau"], None, a["ws"],
+                                    a["ws_bytes"], None)
+    assert cv(idx=None) == 1 and cv(mask=None) == 1 and cv(ws=None) == 1
+    assert cv(K=0) == 2 and cv(K=V + 1) == 2 and cv(tau=-1.0) == 2 and cv(N=-1) == 2
+    assert cv(idx=0x30002) == 3 and cv(ws=0x80040) == 3
+    assert cv(ws_bytes=need // 2) == 5 and "workspace" in K.kdkl_last_error()
+    # the workspace layout does not depend on d, so the count's workspace serves the forward and backward
+    assert need == K.kdkl_workspace_bytes(N, 4096, V, Kc)

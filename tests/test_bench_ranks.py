@@ -71,12 +71,14 @@ def test_reference_arm_prints_contract_line(steps, capsys, monkeypatch):
 
 
 def test_reference_arm_counts_the_rows_it_times():
-    """The oracle sample never exceeds the workload's N rows, and the rate is computed from
-    the rows actually processed (the tiny workload has 256)."""
+    """Each step times one seeded sample of bench.CPU_SAMPLE_ROWS rows (the GPU line's
+    cpu_baseline times the same sample size), and the rate is computed from the rows
+    actually processed."""
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "tiny",
                           "--steps", "2", "--warmup", "0"], capture_output=True, text=True, timeout=300, cwd=ROOT)
     assert out.returncode == 0, out.stderr
     line = json.loads(out.stdout.strip().splitlines()[-1])
-    assert line["config"]["sample_rows_per_step"] == 256
-    assert line["cpu_baseline"]["sample"].startswith("256 seeded rows")
-    assert abs(line["value"] - 256 * 2 / (line["ms_per_step"] * 2 / 1000.0)) <= 1e-6 * line["value"]
+    n = min(bench.CPU_SAMPLE_ROWS, synth.CONFIGS["tiny"].N)
+    assert line["config"]["sample_rows_per_step"] == n
+    assert line["cpu_baseline"]["sample"].startswith(f"{n} seeded rows")
+    assert abs(line["value"] - n * 2 / (line["ms_per_step"] * 2 / 1000.0)) <= 1e-6 * line["value"]

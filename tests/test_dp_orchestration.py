@@ -19,21 +19,27 @@ from output_head_kl_b200 import dp
 
 
 class OracleOps:
-    """Stand-in for the kernels: the oracle on this rank's shard, same normalisation contract."""
+    """Stand-in for the kernels: the oracle on this rank's shard, same contract as the
+    library (count; loss and gradients normalised by the count passed in)."""
 
     def __init__(self, x):
         self.x = x
 
-    def forward(self, hidden, W, idx, logit, mask, tau):
+    def count(self, hidden, W, idx, logit, mask, tau):
         r = O.kl_loss(self.x.hidden_bits, self.x.W_bits, self.x.topk_idx, self.x.topk_logit, self.x.mask, tau,
                       want_grads=False)
         self.nv = r.n_valid
-        return (torch.tensor([r.loss], dtype=torch.float64), torch.tensor(r.lse),
-                torch.tensor([r.n_valid], dtype=torch.int32), None)
+        return torch.tensor([r.n_valid], dtype=torch.int32), None
+
+    def forward(self, hidden, W, idx, logit, mask, tau, ws, n_valid_global):
+        r = O.kl_loss(self.x.hidden_bits, self.x.W_bits, self.x.topk_idx, self.x.topk_logit, self.x.mask, tau,
+                      want_grads=False)
+        scale = (self.nv / int(n_valid_global.item())) if self.nv else 0.0   # the oracle uses the local count
+        return torch.tensor([r.loss * scale], dtype=torch.float64), torch.tensor(r.lse)
 
     def backward(self, hidden, W, idx, logit, mask, tau, lse, ws, n_valid_global):
         r = O.kl_loss(self.x.hidden_bits, self.x.W_bits, self.x.topk_idx, self.x.topk_logit, self.x.mask, tau)
-        scale = (self.nv / int(n_valid_global.item())) if self.nv else 0.0   # oracle grads use the local count
+        scale = (self.nv / int(n_valid_global.item())) if self.nv else 0.0
         return torch.tensor(r.dH * scale), torch.tensor(r.dW * scale)
 
 

@@ -121,3 +121,29 @@ def test_global_normaliser_option_and_dp_step_single_rank():
     assert int(res.n_valid_global.item()) == nv
     assert res.loss.item() == pytest.approx(base.loss, rel=1e-6)
     np.testing.assert_array_equal(res.dW.cpu().numpy(), base.dW.astype(np.float32))
+
+
+def test_count_valid_matches_the_oracle_count_and_flags():
+    """kdkl_count_valid leaves the oracle's N_valid (rows with a NaN logit or no in-range
+    entry are not counted) at kdkl_n_valid_device, with the data-error flags; the forward on
+    the same workspace then reports the same count."""
+    N, d, V, Kc = 300, 64, 1000, 8
+    x = synth.custom_inputs(N, d, V, Kc, seed=309, mask_frac=0.1, w_std=0.1)
+    x.mask[5] = x.mask[7] = 1
+    x.topk_logit[5, 2] = np.nan          # a non-finite teacher row: treated as masked
+    x.topk_idx[7, :] = -1                # no in-range entry: treated as masked
+    dx = H.to_device(x)
+    ws = torch.empty(K.kdkl_workspace_bytes(N, d, V, Kc), dtype=torch.uint8, device="cuda")
+    K.kdkl_count_valid(dx.idx, dx.logit, dx.mask, dx.tau, V, ws)
+    count = K.n_valid_view(ws)
+    nv = int(count.item())
+    flags = K.kdkl_read_device_flags(ws)
+    r = O.kl_loss(x.hidden_bits, x.W_bits, x.topk_idx, x.topk_logit, x.mask, x.tau, want_grads=False)
+    assert nv == r.n_valid == int((x.mask != 0).sum()) - 2
+    assert flags == r.flags == (K.DEV_IDX_RANGE | K.DEV_NONFINITE)
+    loss = torch.empty(1, device="cuda")
+    lse = torch.empty(N, device="cuda")
+    K.kdkl_forward(dx.hidden, dx.W, dx.idx, dx.logit, dx.mask, dx.tau, loss, lse, ws)
+    assert int(count.item()) == nv
+    K.kdkl_count_valid(dx.idx, dx.logit, dx.mask, dx.tau, V, ws, N=0)
+    assert int(count.item()) == 0
