@@ -111,8 +111,9 @@ def record_traffic(csv_path: str, workload: str) -> dict:
     rec = json.load(open(p)) if os.path.exists(p) else {}
     if rec.get("sources_sha256") != kernel_sources_digest():
         rec = {"sources_sha256": kernel_sources_digest(), "workloads": {}}
-    rec["workloads"][workload] = {k: {"dram_bytes_per_launch": sum(v) / len(v), "launches_captured": len(v)}
-                                  for k, v in sums.items()}
+    # kernels captured in separate runs (the forward, the backward chunk) merge into one entry
+    rec["workloads"].setdefault(workload, {}).update(
+        {k: {"dram_bytes_per_launch": sum(v) / len(v), "launches_captured": len(v)} for k, v in sums.items()})
     with open(p, "w") as f:
         json.dump(rec, f, indent=1, sort_keys=True)
     return rec

@@ -44,7 +44,10 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 constexpr int64_t kDefaultChunk = 8192;
-constexpr int kDefaultSyncWindow = 4;
+constexpr int kDefaultSyncWindow = 1;      // row-stream GEMMs: tiles (measured best of 0, 1, 2, 4, 8)
+constexpr int kDefaultSyncKWindow = 32;    // tile-mode GEMMs: reduction blocks
+constexpr int kSplitGroupMB = 32;          // split-major GEMMs: hidden rows per row-block group
+constexpr int kTileColGroup = 0;           // dHidden / dW: column tiles per group (0 = all)
 constexpr int64_t kMaxRows = (int64_t(1) << 31) - 256;
 constexpr int32_t kMaxV = (int32_t(1) << 30);
 
@@ -439,17 +442,42 @@ EpiParams base_params(const Common& c, const WsLayout& L) {
   return ep;
 }
 
-// Tiles a group may run ahead of the slowest group sharing its vocabulary split
-// (the lockstep of the row-stream GEMMs; 0 = off).  KDKL_SYNC_WINDOW overrides the
-// default, for tuning.
+// How far a group may run ahead of the slowest group sharing its operands (the
+// lockstep; 0 = off): in tiles for the row-stream GEMMs, in 64-wide reduction blocks
+// for the tile-mode ones.  KDKL_SYNC_WINDOW / KDKL_SYNC_KWINDOW override the defaults,
+// for tuning.
+int env_window(const char* name, int dflt) {
+  const char* e = std::getenv(name);
+  int v = dflt;
+  if (e && *e) v = std::atoi(e);
+  return v < 0 ? 0 : v;
+}
 int sync_window() {
-  static int w = [] {
-    const char* e = std::getenv("KDKL_SYNC_WINDOW");
-    int v = kDefaultSyncWindow;
-    if (e && *e) v = std::atoi(e);
-    return v < 0 ? 0 : v;
-  }();
+  static int w = env_window("KDKL_SYNC_WINDOW", kDefaultSyncWindow);
   return w;
+}
+int sync_kwindow() {
+  static int w = env_window("KDKL_SYNC_KWINDOW", kDefaultSyncKWindow);
+  return w;
+}
+
+// Row blocks per group of a split-major launch: about kSplitGroupBytes of hidden rows
+// (KDKL_SPLIT_GROUP_MB overrides it for tuning; 0 = one group of every row block).
+// Every group streams all of W once, so smaller groups trade W passes for fewer hidden
+// rows that must stay in L2 while each W tile is shared.
+// Column tiles per group of the dHidden / dW launches (KDKL_TILE_COL_GROUP, for tuning;
+// 0 = all tiles of a row block in a row).
+int tile_col_group() {
+  static int g = env_window("KDKL_TILE_COL_GROUP", kTileColGroup);
+  return g;
+}
+
+int split_rb_group(int d, int rows_per_block) {
+  static int mb = env_window("KDKL_SPLIT_GROUP_MB", kSplitGroupMB);
+  if (mb <= 0) return 0;
+  const double rows_bytes = static_cast<double>(rows_per_block) * d * 2.0;
+  const int g = static_cast<int>(mb * 1048576.0 / rows_bytes);
+  return g < 1 ? 1 : g;
 }
 
 // L2 eviction priorities of the operand loads (KDKL_L2_HINTS, a bit mask, for tuning;
@@ -465,14 +493,14 @@ int l2_hint_mask() {
   return m;
 }
 
-// Arms the lockstep of a row-stream launch of `grid` CTAs: clears the groups'
-// position words on the stream, ahead of the launch.
+// Arms the lockstep of a launch of `grid` CTAs: clears the groups' position words on
+// the stream, ahead of the launch.
 cudaError_t arm_sync(Sched& sc, unsigned long long* prog, int grid, bool pair, cudaStream_t s) {
   const int groups = pair ? grid / 2 : grid;
   sc.sync_window = 0;
   sc.prog = prog;
-  if (l2_hint_mask() & 1) sc.l2_a = kL2Last;
-  const int w = sync_window();
+  if (sc.row_stream && (l2_hint_mask() & 1)) sc.l2_a = kL2Last;
+  const int w = sc.row_stream ? sync_window() : sync_kwindow();
   if (w <= 0 || groups > kSyncSlots || groups < 2) return cudaSuccess;
   sc.sync_window = w;
   return cudaMemsetAsync(prog, 0, static_cast<size_t>(groups) * 8, s);
@@ -630,12 +658,13 @@ kdkl_status kdkl_forward_ex(const void* hidden, const void* W, const void* topk_
 static kdkl_status run_dh_dw(const EpiParams& ep0, const Pairing& pd, int bn, int32_t V, int32_t d, int64_t c0,
                              int64_t nc, const CUtensorMap& tmG_k, const CUtensorMap& tmG_mn,
                              const CUtensorMap& tmW_mn, const CUtensorMap& tmH_mn, void* dHidden, float* dW,
-                             cudaStream_t s) {
+                             unsigned long long* prog, cudaStream_t s) {
   const int nt = (d + bn - 1) / bn;
   cudaError_t e;
   {
     const int64_t rbc = (nc + pd.rows - 1) / pd.rows;
     Sched sc{static_cast<int>(rbc * nt), 1, nt, static_cast<int>((V + kBK - 1) / kBK), 0};
+    sc.col_group = tile_col_group();
     EpiParams ep = ep0;
     ep.M = static_cast<int>(nc);
     ep.Ncols = d;
@@ -643,6 +672,7 @@ static kdkl_status run_dh_dw(const EpiParams& ep0, const Pairing& pd, int bn, in
     ep.dH = static_cast<uint16_t*>(dHidden);
     ep.ldo = d;
     const int grid = pd.grid(sc.units);
+    if ((e = arm_sync(sc, prog, grid, pd.pair, s)) != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
     if ((e = timed(kTDh, s, [&] {
            return launch_gemm(kEpiStoreBf16, bn, pd.pair, tmG_k, tmW_mn, tmG_k, sc, ep, grid, s);
          })) != cudaSuccess)
@@ -651,6 +681,7 @@ static kdkl_status run_dh_dw(const EpiParams& ep0, const Pairing& pd, int bn, in
   {
     const int64_t vb = (V + pd.rows - 1) / pd.rows;
     Sched sc{static_cast<int>(vb * nt), 1, nt, static_cast<int>((nc + kBK - 1) / kBK), 0};
+    sc.col_group = tile_col_group();
     if (l2_hint_mask() & 2) sc.l2_b = kL2Last;
     EpiParams ep = ep0;
     ep.M = V;
@@ -665,6 +696,7 @@ static kdkl_status run_dh_dw(const EpiParams& ep0, const Pairing& pd, int bn, in
     if (!make_map_f32(&tmDW, dW, d, V, d, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B))
       return fail(KDKL_ERR_CUDA, "cuTensorMapEncodeTiled failed (dW)");
     const int grid = pd.grid(sc.units);
+    if ((e = arm_sync(sc, prog, grid, pd.pair, s)) != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
     if ((e = timed(kTDw, s, [&] {
            return launch_gemm(kEpiRmwF32, bn, pd.pair, tmG_mn, tmH_mn, tmDW, sc, ep, grid, s);
          })) != cudaSuccess)
@@ -732,6 +764,7 @@ static kdkl_status backward_impl(const void* hidden, const void* W, const void* 
       const int splits = pick_splits(rbc, vt, pg.groups, d, L.units_cap * kBM / pg.rows, pg.rows);
       // a chunk's hidden rows fit in L2, so all its row blocks sweep each split together
       Sched sc{static_cast<int>(rbc * splits), splits, vt, (d + kBK - 1) / kBK, kSplitMajor};
+      sc.rb_group = split_rb_group(d, pg.rows);
       EpiParams ep = ep0;
       ep.M = static_cast<int>(nc);
       ep.Ncols = V;
@@ -745,7 +778,8 @@ static kdkl_status backward_impl(const void* hidden, const void* W, const void* 
         return cuda_fail(e, "gradient GEMM launch");
     }
     // (2) dHidden rows of the chunk = G W; (3) dW (+)= G^T hidden_chunk
-    if ((st = run_dh_dw(ep0, pd, bn, V, d, c0, nc, tmG_k, tmG_mn, tmW_mn, tmH_mn, dHidden, dW, s)) != KDKL_OK)
+    if ((st = run_dh_dw(ep0, pd, bn, V, d, c0, nc, tmG_k, tmG_mn, tmW_mn, tmH_mn, dHidden, dW,
+                        at<unsigned long long>(workspace, L.sync), s)) != KDKL_OK)
       return st;
   }
   return ok();
@@ -837,6 +871,7 @@ static kdkl_status forward_backward_impl(const void* hidden, const void* W, cons
     const int splits = pick_splits(rbc, vt, pg.groups, d, L.units_cap * kBM / pg.rows, pg.rows);
     {
       Sched sc{static_cast<int>(rbc * splits), splits, vt, (d + kBK - 1) / kBK, kSplitMajor};
+      sc.rb_group = split_rb_group(d, pg.rows);
       EpiParams ep = ep0;
       ep.M = static_cast<int>(nc);
       ep.Ncols = V;
@@ -869,7 +904,8 @@ static kdkl_status forward_backward_impl(const void* hidden, const void* W, cons
          })) != cudaSuccess)
       return cuda_fail(e, "G launch");
     // (4) dHidden rows of the chunk = G W; (5) dW (+)= G^T hidden_chunk
-    if ((st = run_dh_dw(ep0, pd, bn, V, d, c0, nc, tmG_k, tmG_mn, tmW_mn, tmH_mn, dHidden, dW, s)) != KDKL_OK)
+    if ((st = run_dh_dw(ep0, pd, bn, V, d, c0, nc, tmG_k, tmG_mn, tmW_mn, tmH_mn, dHidden, dW,
+                        at<unsigned long long>(workspace, L.sync), s)) != KDKL_OK)
       return st;
   }
   return ok();

@@ -47,12 +47,15 @@ WsLayout make_layout(int64_t N, int32_t d, int32_t V, int32_t K, int64_t chunk_t
 //     [(j * n_tiles) / splits, ((j + 1) * n_tiles) / splits) with j = u % splits.
 //   tile mode: unit u -> row block u / n_tiles, the single tile u % n_tiles.
 // Work units of a persistent GEMM launch, dealt round-robin to the CTA groups.
-//   row_stream = 0: one output tile per unit, u = row block * n_tiles + tile;
+//   row_stream = 0: one output tile per unit, u = row block * n_tiles + tile, or with
+//     col_group > 0 the tiles in groups of col_group columns, each group swept row
+//     block by row block (fewer B columns in flight at once, more passes over A);
 //   row_stream = kRowMajor: a unit is (row block, vocabulary split) and sweeps the
 //     split's tiles, u = row block * splits + split (the row blocks in flight stay few);
-//   row_stream = kSplitMajor: the same units, u = split * row blocks + row block, so
-//     the groups running at once cover every row block of one split and share its
-//     W tiles (for launches whose row blocks all fit in L2).
+//   row_stream = kSplitMajor: the same units, dealt in groups of rb_group row blocks
+//     (0 = all of them): within a group u = split * rows of the group + row block, so
+//     the CTA groups running at once cover every row block of the group for one split
+//     and share its W tiles, while only the group's hidden rows need to stay in L2.
 constexpr int kRowMajor = 1;
 constexpr int kSplitMajor = 2;
 //
@@ -60,14 +63,18 @@ constexpr int kSplitMajor = 2;
 // the same vocabulary split in the same round (round k = units [k G, k G + G) for G
 // groups; group g runs unit g + k G) stream the same W tiles, which only one DRAM
 // read serves while they stay close together.  Each group publishes its position
-// (unit + 1) << 32 | (tile - first tile of the unit) in prog[group] as it starts a
-// tile, and the even CTA's producer holds back tile r of a unit until every peer
-// group of that round and split has reached tile r - sync_window.  prog must be
+// (unit + 1) << 32 | (tile - first tile of the unit) in prog[group] as it reaches a
+// tile, and the even CTA's producer then holds back tile r of a unit until every peer
+// group of that round and split has reached tile r - sync_window.  Tile-mode launches
+// (dHidden, dW: one long reduction per unit, and the units of a round share rows of A
+// or columns of B) do the same every kSyncKStep reduction blocks, with every unit of
+// the round as a peer and sync_window counted in reduction blocks.  prog must be
 // zeroed before the launch.  A wait that lasts longer than kSyncSoftLimitNs gives
 // up and the group stops holding back for the rest of its unit; waiting never
 // changes results, only how far the groups drift apart.
 enum L2Priority { kL2Normal = 0, kL2Last = 1, kL2First = 2 };
 constexpr int kSyncSlots = 1024;                          // groups a synchronised launch may have
+constexpr int kSyncKStep = 16;                            // tile mode: reduction blocks per position step
 constexpr unsigned long long kSyncSoftLimitNs = 1000000;  // 1 ms
 struct Sched {
   int units;
@@ -80,6 +87,8 @@ struct Sched {
   // L2 eviction priority of the A and B operand loads (kL2Normal = 0, kL2Last, kL2First)
   int l2_a;
   int l2_b;
+  int rb_group;   // kSplitMajor: row blocks per group (0 = all)
+  int col_group;  // tile mode: column tiles per group (0 = all; u = row block * n_tiles + tile)
 };
 
 // Parameters of the fused epilogues (the union of what each kind needs).

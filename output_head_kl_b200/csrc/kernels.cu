@@ -391,9 +391,15 @@ __device__ __forceinline__ void unit_range(const Sched& sc, int u, int& mb, int&
   j = 0;
   if (sc.row_stream) {
     if (sc.row_stream == kSplitMajor) {
+      // groups of rb_group row blocks, each swept split by split; the last group may
+      // hold fewer row blocks
       const int rb = sc.units / sc.splits;
-      j = u / rb;
-      mb = u - j * rb;
+      const int gsz = (sc.rb_group > 0 && sc.rb_group < rb) ? sc.rb_group : rb;
+      const int g = u / (gsz * sc.splits);
+      const int rbg = min(gsz, rb - g * gsz);
+      const int off = u - g * gsz * sc.splits;
+      j = off / rbg;
+      mb = g * gsz + (off - j * rbg);
     } else {
       mb = u / sc.splits;
       j = u - mb * sc.splits;
@@ -401,30 +407,49 @@ __device__ __forceinline__ void unit_range(const Sched& sc, int u, int& mb, int&
     t0 = static_cast<int>((static_cast<int64_t>(j) * sc.n_tiles) / sc.splits);
     t1 = static_cast<int>((static_cast<int64_t>(j + 1) * sc.n_tiles) / sc.splits);
   } else {
-    mb = u / sc.n_tiles;
-    t0 = u - mb * sc.n_tiles;
+    // groups of col_group column tiles (0 = all), each swept row block by row block;
+    // the last group may hold fewer tiles
+    const int rows = sc.units / sc.n_tiles;
+    const int cg = (sc.col_group > 0 && sc.col_group < sc.n_tiles) ? sc.col_group : sc.n_tiles;
+    const int g = u / (rows * cg);
+    const int cgs = min(cg, sc.n_tiles - g * cg);
+    const int off = u - g * rows * cg;
+    mb = off / cgs;
+    t0 = g * cg + (off - mb * cgs);
     t1 = t0 + 1;
   }
 }
 
-// Position word a group publishes as it starts relative tile r of unit u.
+// Position word a group publishes as it reaches position r of unit u (the relative tile
+// of a row-stream unit, the reduction block of a tile-mode unit).
 __device__ __forceinline__ unsigned long long sync_word(int u, int r) {
   return (static_cast<unsigned long long>(u + 1) << 32) | static_cast<unsigned int>(r);
 }
 
-// Whole warp (the producer warp of an even CTA): the smallest relative tile that the
-// other groups running a unit of split j in unit u's round have reached in that unit
-// (a peer already past that unit counts as INT_MAX, one not yet in it as -1), waiting
-// until it is at least r_need.  Returns -2 if the wait gave up (kSyncSoftLimitNs).
+// Whole warp (the producer warp of an even CTA): the smallest position that the peers
+// of unit u have reached in their units (a peer already past its unit counts as
+// INT_MAX, one not yet in it as -1), waiting until it is at least r_need.  The peers
+// are the other units of u's round that stream the same operand: those of vocabulary
+// split j (row-stream launches), or every unit of the round (tile-mode launches, whose
+// units share rows of A or columns of B).  Returns -2 if the wait gave up
+// (kSyncSoftLimitNs).
 __device__ int wait_split_peers(const Sched& sc, int u, int group, int ngroups, int j, int r_need, int lane,
                                 uint32_t* flags) {
   const int round0 = u - group;                  // group g runs units g + k G: this round is [k G, k G + G)
   const int round1 = min(round0 + ngroups, sc.units);
   int first, last, step;
-  if (sc.row_stream == kSplitMajor) {            // units of split j are j rb ... j rb + rb - 1
+  if (sc.row_stream == 0) {                      // tile mode: the whole round
+    first = round0;
+    last = round1;
+    step = 1;
+  } else if (sc.row_stream == kSplitMajor) {     // split j of u's row-block group: contiguous units
     const int rb = sc.units / sc.splits;
-    first = max(round0, j * rb);
-    last = min(round1, (j + 1) * rb);
+    const int gsz = (sc.rb_group > 0 && sc.rb_group < rb) ? sc.rb_group : rb;
+    const int g = u / (gsz * sc.splits);
+    const int rbg = min(gsz, rb - g * gsz);
+    const int gbase = g * gsz * sc.splits;
+    first = max(round0, gbase + j * rbg);
+    last = min(round1, gbase + (j + 1) * rbg);
     step = 1;
   } else {                                       // units of split j are those with u % splits == j
     first = round0 + ((j - round0 % sc.splits) % sc.splits + sc.splits) % sc.splits;
@@ -551,7 +576,10 @@ __global__ void __launch_bounds__(192, 1)
     uint32_t phase = 0;
     bool wrapped = false;    // every stage has been filled at least once
     bool stop = false;
-    const bool sync_on = sc.sync_window > 0 && sc.row_stream != 0 && rank == 0;
+    const bool sync_on = sc.sync_window > 0 && rank == 0;
+    // row-stream units synchronise per tile; tile-mode units (one long reduction each)
+    // per segment of kSyncKStep reduction blocks
+    const int kseg = (sync_on && sc.row_stream == 0) ? kSyncKStep : sc.k_blocks;
     const bool hints = (sc.l2_a | sc.l2_b) != 0;
     const uint64_t pol_a = l2_policy(sc.l2_a), pol_b = l2_policy(sc.l2_b);
     for (int u = group; u < sc.units && !stop; u += ngroups) {
@@ -559,85 +587,92 @@ __global__ void __launch_bounds__(192, 1)
       unit_range(sc, u, mb, uj, t0, t1);
       const int arow = mb * C::kMmaM + static_cast<int>(rank) * kBM;   // this CTA's A rows
       bool hold = sync_on;
-      int seen = -1;          // every peer had reached this relative tile at the last look
+      int seen = -1;          // every peer had reached this position at the last look
       for (int t = t0; t < t1 && !stop; ++t) {
-        if (sync_on) {
-          const int need = t - t0 - sc.sync_window;
-          if (hold && need > seen) {
-            const int got = wait_split_peers(sc, u, group, ngroups, uj, need, lane, ep.flags);
-            if (got == -2) hold = false;
-            else seen = got;
-          }
-          if (lane == 0) *reinterpret_cast<volatile unsigned long long*>(sc.prog + group) = sync_word(u, t - t0);
-        }
-        int lstop = 0;
-        if (lane == 0) {
-          int bcol = t * BN + static_cast<int>(rank) * C::kCtaN;  // this CTA's B rows (N)
-          if (C::kBmn && !dbg_ok((bcol & 7) == 0, ep.flags)) bcol &= ~7;   // x of an MN-major bf16 box
-          for (int kb = 0; kb < sc.k_blocks; ++kb) {
-            if (!mbar_wait(&empty[stage], phase ^ 1u, ab)) {
-              lstop = 1;
-              break;
+        int bcol = t * BN + static_cast<int>(rank) * C::kCtaN;  // this CTA's B rows (N)
+        if (C::kBmn && !dbg_ok((bcol & 7) == 0, ep.flags)) bcol &= ~7;   // x of an MN-major bf16 box
+        for (int kb0 = 0; kb0 < sc.k_blocks && !stop; kb0 += kseg) {
+          if (sync_on) {
+            // publish first, then wait: every peer has then published at least the
+            // position it waits at, so the slowest peer's condition always holds
+            const int pos = sc.row_stream ? t - t0 : kb0;
+            const int need = pos - sc.sync_window;
+            if (lane == 0) *reinterpret_cast<volatile unsigned long long*>(sc.prog + group) = sync_word(u, pos);
+            __syncwarp();
+            if (hold && need > seen) {
+              const int got = wait_split_peers(sc, u, group, ngroups, uj, need, lane, ep.flags);
+              if (got == -2) hold = false;
+              else seen = got;
             }
-            uint8_t* a = sA + stage * C::kABytes;
-            uint8_t* b = sB + stage * C::kBBytes;
-            if (PAIR) {
-              // both CTAs' bytes are counted on the even CTA's barrier
-              const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
-              if (rank == 0) mbar_arrive_expect_tx(&full[stage], C::kTxBytes);
-              if (hints) {
-                if (C::kAmn) {
-                  tma_load_2d_pair_hint(a, &tmA, bar0, arow, kb * kBK, pol_a);
-                  tma_load_2d_pair_hint(a + 8192, &tmA, bar0, arow + 64, kb * kBK, pol_a);
+          }
+          int lstop = 0;
+          if (lane == 0) {
+            const int kb1 = min(kb0 + kseg, sc.k_blocks);
+            for (int kb = kb0; kb < kb1; ++kb) {
+              if (!mbar_wait(&empty[stage], phase ^ 1u, ab)) {
+                lstop = 1;
+                break;
+              }
+              uint8_t* a = sA + stage * C::kABytes;
+              uint8_t* b = sB + stage * C::kBBytes;
+              if (PAIR) {
+                // both CTAs' bytes are counted on the even CTA's barrier
+                const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
+                if (rank == 0) mbar_arrive_expect_tx(&full[stage], C::kTxBytes);
+                if (hints) {
+                  if (C::kAmn) {
+                    tma_load_2d_pair_hint(a, &tmA, bar0, arow, kb * kBK, pol_a);
+                    tma_load_2d_pair_hint(a + 8192, &tmA, bar0, arow + 64, kb * kBK, pol_a);
+                  } else {
+                    tma_load_2d_pair_hint(a, &tmA, bar0, kb * kBK, arow, pol_a);
+                  }
+                  if (C::kBmn) {
+#pragma unroll
+                    for (int q = 0; q < C::kBAtoms; ++q)
+                      tma_load_2d_pair_hint(b + q * 8192, &tmB, bar0, bcol + q * 64, kb * kBK, pol_b);
+                  } else {
+                    tma_load_2d_pair_hint(b, &tmB, bar0, kb * kBK, bcol, pol_b);
+                  }
                 } else {
-                  tma_load_2d_pair_hint(a, &tmA, bar0, kb * kBK, arow, pol_a);
+                  if (C::kAmn) {
+                    tma_load_2d_pair(a, &tmA, bar0, arow, kb * kBK);
+                    tma_load_2d_pair(a + 8192, &tmA, bar0, arow + 64, kb * kBK);
+                  } else {
+                    tma_load_2d_pair(a, &tmA, bar0, kb * kBK, arow);
+                  }
+                  if (C::kBmn) {
+#pragma unroll
+                    for (int q = 0; q < C::kBAtoms; ++q)
+                      tma_load_2d_pair(b + q * 8192, &tmB, bar0, bcol + q * 64, kb * kBK);
+                  } else {
+                    tma_load_2d_pair(b, &tmB, bar0, kb * kBK, bcol);
+                  }
+                }
+              } else {
+                mbar_arrive_expect_tx(&full[stage], C::kTxBytes);
+                if (C::kAmn) {
+                  tma_load_2d(a, &tmA, &full[stage], arow, kb * kBK);
+                  tma_load_2d(a + 8192, &tmA, &full[stage], arow + 64, kb * kBK);
+                } else {
+                  tma_load_2d(a, &tmA, &full[stage], kb * kBK, arow);
                 }
                 if (C::kBmn) {
 #pragma unroll
                   for (int q = 0; q < C::kBAtoms; ++q)
-                    tma_load_2d_pair_hint(b + q * 8192, &tmB, bar0, bcol + q * 64, kb * kBK, pol_b);
+                    tma_load_2d(b + q * 8192, &tmB, &full[stage], bcol + q * 64, kb * kBK);
                 } else {
-                  tma_load_2d_pair_hint(b, &tmB, bar0, kb * kBK, bcol, pol_b);
-                }
-              } else {
-                if (C::kAmn) {
-                  tma_load_2d_pair(a, &tmA, bar0, arow, kb * kBK);
-                  tma_load_2d_pair(a + 8192, &tmA, bar0, arow + 64, kb * kBK);
-                } else {
-                  tma_load_2d_pair(a, &tmA, bar0, kb * kBK, arow);
-                }
-                if (C::kBmn) {
-#pragma unroll
-                  for (int q = 0; q < C::kBAtoms; ++q)
-                    tma_load_2d_pair(b + q * 8192, &tmB, bar0, bcol + q * 64, kb * kBK);
-                } else {
-                  tma_load_2d_pair(b, &tmB, bar0, kb * kBK, bcol);
+                  tma_load_2d(b, &tmB, &full[stage], kb * kBK, bcol);
                 }
               }
-            } else {
-              mbar_arrive_expect_tx(&full[stage], C::kTxBytes);
-              if (C::kAmn) {
-                tma_load_2d(a, &tmA, &full[stage], arow, kb * kBK);
-                tma_load_2d(a + 8192, &tmA, &full[stage], arow + 64, kb * kBK);
-              } else {
-                tma_load_2d(a, &tmA, &full[stage], kb * kBK, arow);
+              if (++stage == C::kStages) {
+                stage = 0;
+                phase ^= 1u;
+                wrapped = true;
               }
-              if (C::kBmn) {
-#pragma unroll
-                for (int q = 0; q < C::kBAtoms; ++q)
-                  tma_load_2d(b + q * 8192, &tmB, &full[stage], bcol + q * 64, kb * kBK);
-              } else {
-                tma_load_2d(b, &tmB, &full[stage], kb * kBK, bcol);
-              }
-            }
-            if (++stage == C::kStages) {
-              stage = 0;
-              phase ^= 1u;
-              wrapped = true;
             }
           }
+          stop = __shfl_sync(0xffffffffu, lstop, 0) != 0;
         }
-        stop = __shfl_sync(0xffffffffu, lstop, 0) != 0;
       }
     }
     if (lane == 0 && rank == 0 && *abort_flag) {
