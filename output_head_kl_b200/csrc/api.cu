@@ -45,7 +45,7 @@ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_
 
 constexpr int64_t kDefaultChunk = 8192;
 constexpr int kDefaultSyncWindow = 1;      // row-stream GEMMs: tiles (measured best of 0, 1, 2, 4, 8)
-constexpr int kDefaultSyncKWindow = 32;    // tile-mode GEMMs: reduction blocks
+constexpr int kDefaultSyncKWindow = 64;    // tile-mode GEMMs: reduction blocks (measured best of 0, 8 ... 256)
 constexpr int kSplitGroupMB = 32;          // split-major GEMMs: hidden rows per row-block group
 constexpr int kTileColGroup = 0;           // dHidden / dW: column tiles per group (0 = all)
 constexpr int64_t kMaxRows = (int64_t(1) << 31) - 256;
@@ -114,6 +114,14 @@ kdkl_status current_device(Device& dv) {
   return KDKL_OK;
 }
 
+// A tuning knob: the environment variable `name` as a non-negative integer, or dflt.
+int env_window(const char* name, int dflt) {
+  const char* e = std::getenv(name);
+  int v = dflt;
+  if (e && *e) v = std::atoi(e);
+  return v < 0 ? 0 : v;
+}
+
 // Vocabulary splits for a row-stream kernel over `rb` row blocks and `vt`
 // vocabulary tiles: balance the per-group tile count over `ctas` CTA groups
 // (single CTAs or CTA pairs), and keep at least enough splits that the hidden
@@ -123,9 +131,11 @@ int pick_splits(int64_t rb, int vt, int ctas, int d, int64_t units_cap, int rows
   // but more hidden rows in flight.  Measured on B200 (forward, steady state):
   // the fastest split counts were 2 at (N, d, V) = (131072, 2880, 201088),
   // 3 at (131072, 4096, 128256) and 4 at (32768, 4096, 128256), i.e. 37-55 MB of
-  // hidden rows in flight, 3-9 % faster than at 18-20 MB.
+  // hidden rows in flight, 3-9 % faster than at 18-20 MB.  KDKL_ROWS_BUDGET_MB
+  // overrides the budget, for tuning.
   const double rows_bytes = static_cast<double>(rows_per_block) * d * 2.0;
-  const double budget = 55.0 * 1024 * 1024;
+  static const int budget_mb = env_window("KDKL_ROWS_BUDGET_MB", 55);   // override for tuning
+  const double budget = budget_mb * 1024.0 * 1024.0;
   int s_min = static_cast<int>(std::ceil(ctas * rows_bytes / budget));
   if (s_min < s_floor) s_min = s_floor;
   if (s_min < 1) s_min = 1;
@@ -446,12 +456,6 @@ EpiParams base_params(const Common& c, const WsLayout& L) {
 // lockstep; 0 = off): in tiles for the row-stream GEMMs, in 64-wide reduction blocks
 // for the tile-mode ones.  KDKL_SYNC_WINDOW / KDKL_SYNC_KWINDOW override the defaults,
 // for tuning.
-int env_window(const char* name, int dflt) {
-  const char* e = std::getenv(name);
-  int v = dflt;
-  if (e && *e) v = std::atoi(e);
-  return v < 0 ? 0 : v;
-}
 int sync_window() {
   static int w = env_window("KDKL_SYNC_WINDOW", kDefaultSyncWindow);
   return w;

@@ -786,6 +786,7 @@ __global__ void __launch_bounds__(192, 1)
       uint16_t* hi = reinterpret_cast<uint16_t*>(wbuf_all + kTopKMax * kBM * 4) + row_local;
       const int ubase = t0 * BN;
       float hroot = -INFINITY;
+      int hcnt = 0;   // entries kept so far (the heap fills before its root becomes a threshold)
       if (KIND == kEpiTopK) {
         for (int k = 0; k < ep.topk_K; ++k) {
           hv[k * kBM] = -INFINITY;
@@ -965,10 +966,26 @@ __global__ void __launch_bounds__(192, 1)
               const int j = __ffs(cand) - 1;
               cand &= cand - 1u;
               const float val = pick32(v, static_cast<uint32_t>(j));
-              if (val > hroot) {
-                // replace the root (the smallest kept entry) and sift down; within a
-                // unit columns arrive in increasing order, so ties keep the earlier index
-                const int vi = col + j - ubase;
+              const int vi = col + j - ubase;
+              if (hcnt < Kh) {
+                // still filling: append and sift up.  Within a unit columns arrive in
+                // increasing order, so a later column of equal value ranks lower.
+                int pos = hcnt++;
+                while (pos > 0) {
+                  const int par = (pos - 1) >> 1;
+                  const float pv = hv[par * kBM];
+                  const int pi = hi[par * kBM];
+                  if (pv < val || (pv == val && pi > vi)) break;   // the parent ranks lower
+                  hv[pos * kBM] = pv;
+                  hi[pos * kBM] = static_cast<uint16_t>(pi);
+                  pos = par;
+                }
+                hv[pos * kBM] = val;
+                hi[pos * kBM] = static_cast<uint16_t>(vi);
+                if (hcnt == Kh) hroot = hv[0];
+              } else if (val > hroot) {
+                // replace the root (the smallest kept entry) and sift down; ties keep the
+                // earlier index
                 int pos = 0;
                 while (true) {
                   const int l = 2 * pos + 1;
