@@ -48,6 +48,7 @@ constexpr int kDefaultSyncWindow = 1;      // row-stream GEMMs: tiles (measured 
 constexpr int kDefaultSyncKWindow = 64;    // tile-mode GEMMs: reduction blocks (measured best of 0, 8 ... 256)
 constexpr int kSplitGroupMB = 32;          // split-major GEMMs: hidden rows per row-block group
 constexpr int kTileColGroup = 0;           // dHidden / dW: column tiles per group (0 = all)
+constexpr int kDieOrder = 0;               // GEMM groups numbered by block index
 constexpr int64_t kMaxRows = (int64_t(1) << 31) - 256;
 constexpr int32_t kMaxV = (int32_t(1) << 30);
 
@@ -469,6 +470,13 @@ int sync_kwindow() {
 // (KDKL_SPLIT_GROUP_MB overrides it for tuning; 0 = one group of every row block).
 // Every group streams all of W once, so smaller groups trade W passes for fewer hidden
 // rows that must stay in L2 while each W tile is shared.
+// Group numbering by the half of the SM ids a CTA group runs on (KDKL_DIE_ORDER, for
+// tuning; 0 = by block index).
+int die_order() {
+  static int v = env_window("KDKL_DIE_ORDER", kDieOrder);
+  return v;
+}
+
 // Column tiles per group of the dHidden / dW launches (KDKL_TILE_COL_GROUP, for tuning;
 // 0 = all tiles of a row block in a row).
 int tile_col_group() {
@@ -502,12 +510,16 @@ int l2_hint_mask() {
 cudaError_t arm_sync(Sched& sc, unsigned long long* prog, int grid, bool pair, cudaStream_t s) {
   const int groups = pair ? grid / 2 : grid;
   sc.sync_window = 0;
+  sc.die_order = 0;
   sc.prog = prog;
   if (sc.row_stream && (l2_hint_mask() & 1)) sc.l2_a = kL2Last;
+  if (groups < 2 || groups + 2 > kSyncSlots) return cudaSuccess;
   const int w = sc.row_stream ? sync_window() : sync_kwindow();
-  if (w <= 0 || groups > kSyncSlots || groups < 2) return cudaSuccess;
-  sc.sync_window = w;
-  return cudaMemsetAsync(prog, 0, static_cast<size_t>(groups) * 8, s);
+  sc.sync_window = w > 0 ? w : 0;
+  sc.die_order = die_order();
+  if (sc.sync_window == 0 && sc.die_order == 0) return cudaSuccess;
+  // the groups' position words and, after them, the two ticket counters of die_order
+  return cudaMemsetAsync(prog, 0, static_cast<size_t>(groups + 2) * 8, s);
 }
 
 }  // namespace

@@ -89,6 +89,7 @@ struct Sched {
   int l2_b;
   int rb_group;   // kSplitMajor: row blocks per group (0 = all)
   int col_group;  // tile mode: column tiles per group (0 = all; u = row block * n_tiles + tile)
+  int die_order;  // number the CTA groups by the half of the SM ids they run on (prog[ngroups..+1] = tickets)
 };
 
 // Parameters of the fused epilogues (the union of what each kind needs).

@@ -528,10 +528,10 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* ebar = drain + 1;             // dW epilogue: one load barrier per staging buffer (4 warps x 2)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ebar + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_group = reinterpret_cast<int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;   // 0 = the CTA that issues the MMAs
-  const int group = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
   const int ngroups = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
@@ -546,6 +546,19 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(drain, 1);
     for (int b = 0; b < 8; ++b) mbar_init(&ebar[b], 1);
     *abort_flag = 0;
+    int g = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+    if (sc.die_order && rank == 0) {
+      // Group numbers by die: the groups on the SMs of the lower half of the SM ids take
+      // tickets from 0 upwards, the others from ngroups - 1 downwards, so each half
+      // runs a contiguous range of every round's units.  Exactly ngroups groups take one
+      // ticket each, so the two ranges meet without overlap whatever the halves' sizes.
+      const int die = 2 * static_cast<int>(sm_id()) >= static_cast<int>(sm_count_ids()) ? 1 : 0;
+      const unsigned long long t = atomicAdd(sc.prog + ngroups + die, 1ull);
+      const int tk = static_cast<int>(t);
+      const int gd = die ? ngroups - 1 - tk : tk;
+      if (dbg_ok(gd >= 0 && gd < ngroups, ep.flags)) g = gd;
+    }
+    *s_group = g;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -567,6 +580,8 @@ __global__ void __launch_bounds__(192, 1)
   else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // the pair's group number: the even CTA's (read across the cluster by the odd CTA)
+  const int group = (PAIR && rank != 0) ? ld_shared_cluster_s32(mapa_shared(smem_u32(s_group), 0)) : *s_group;
   const AbortState ab{abort_flag, ep.flags};
 
   if (warp == 0) {
