@@ -42,6 +42,14 @@
  *     the caller reads with kdkl_read_device_flags.  Entries with an index
  *     outside [0, V) are dropped; repeated indices add up; a row with a NaN or
  *     +inf logit, or with no usable entry, is treated as masked.
+ *   - Schedule tuning (not needed for normal use): the environment variables
+ *     KDKL_SYNC_WINDOW, KDKL_SYNC_KWINDOW, KDKL_SPLIT_GROUP_MB,
+ *     KDKL_TILE_COL_GROUP, KDKL_DIE_ORDER and KDKL_L2_HINTS, read once per
+ *     process, change only the order in which the GEMMs' CTA groups take their
+ *     tiles, how closely they are kept together and the L2 priority of their
+ *     loads; every output is bit-identical under any of them.
+ *     KDKL_ROWS_BUDGET_MB changes the forward's vocabulary split count, and so
+ *     the order of each row's log-sum-exp merge (rounding only).
  */
 #ifndef KDKL_H
 #define KDKL_H
