@@ -32,7 +32,10 @@
  *     from the caller's `workspace`.
  *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL
  *     is the legacy default stream).  Nothing synchronises except
- *     kdkl_read_device_flags.  No state is kept between calls.
+ *     kdkl_read_device_flags.  No state is kept between calls.  After one
+ *     eager call on a device, kdkl_forward(_ex), kdkl_backward(_ex) and
+ *     kdkl_forward_backward can be captured in a CUDA graph (every launch and
+ *     memset goes to `stream`); a replay reads the buffers' current contents.
  *   - Argument checks run on the host before any launch; a failed check
  *     returns its status and launches nothing.  kdkl_last_error() then holds a
  *     one-line reason.
