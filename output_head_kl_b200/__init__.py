@@ -8,7 +8,9 @@ raises.
 Names mirror the C entry points: ``kdkl_workspace_bytes``, ``kdkl_forward``,
 ``kdkl_backward``, ``kdkl_forward_ex``, ``kdkl_backward_ex`` (with ``kdkl_options``),
 ``kdkl_forward_noalloc``, ``kdkl_teacher_topk``, ``kdkl_count_valid``, ``kdkl_read_device_flags``, ``kdkl_timing_enable``,
-``kdkl_timing_read``, ``kdkl_status_string``, ``kdkl_last_error``.  ``fused_kl_forward_backward`` is a convenience wrapper
+``kdkl_timing_read``, ``kdkl_status_string``, ``kdkl_last_error``; with the profiling build loaded,
+``kdkl_profile_role_cycles_read`` / ``kdkl_profile_role_cycles_clear`` (``include/kdkl_profile.h``).
+``fused_kl_forward_backward`` is a convenience wrapper
 that allocates the outputs and the workspace with torch (the library itself
 never allocates).
 """
@@ -21,6 +23,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "_lib", "libkdkl.so")
 # The same library with in-kernel index checks (KDKL_DEV_BOUNDS); see build.py.
 DEBUG_LIB_PATH = os.path.join(_HERE, "_lib", "libkdkl_debug.so")
+# The same library with per-role cycle counters in the GEMM kernels; see build.py.
+PROFILE_LIB_PATH = os.path.join(_HERE, "_lib", "libkdkl_prof.so")
 
 KDKL_OK = 0
 STATUS_NAMES = {0: "KDKL_OK", 1: "KDKL_ERR_NULL", 2: "KDKL_ERR_SHAPE", 3: "KDKL_ERR_ALIGN",
@@ -119,6 +123,13 @@ def lib() -> ctypes.CDLL:
     L.kdkl_backward_plan.argtypes = [i64, i32, i32, i32, i64, ctypes.POINTER(Options), i32,
                                      ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int64)]
     L.kdkl_backward_plan.restype = ctypes.c_int
+    if hasattr(L, "kdkl_profile_read_role_cycles"):
+        L.kdkl_profile_role_cycles_shape.argtypes = [ctypes.POINTER(ctypes.c_int32)] * 3
+        L.kdkl_profile_role_cycles_shape.restype = ctypes.c_int
+        L.kdkl_profile_read_role_cycles.argtypes = [vp, sz]
+        L.kdkl_profile_read_role_cycles.restype = ctypes.c_int
+        L.kdkl_profile_clear_role_cycles.argtypes = [vp]
+        L.kdkl_profile_clear_role_cycles.restype = ctypes.c_int
     _lib = L
     return L
 
@@ -372,3 +383,29 @@ def fused_kl_forward_backward(hidden, W, topk_idx, topk_logit, mask, tau, *, gra
     kdkl_backward(hidden, W, topk_idx, topk_logit, mask, tau, lse, grad_loss, dH, dW, workspace,
                   chunk_tokens=chunk_tokens, stream=stream)
     return loss, lse, dH, dW, workspace
+
+
+def _profile_lib() -> ctypes.CDLL:
+    L = lib()
+    if not hasattr(L, "kdkl_profile_read_role_cycles"):
+        raise RuntimeError("the loaded kdkl library is not the profiling build: set LIB_PATH = PROFILE_LIB_PATH "
+                           "before the first call")
+    return L
+
+
+def kdkl_profile_role_cycles_read():
+    """The profiling build's role cycle counters, a numpy uint64 array [kind, cta, slot]
+    (see include/kdkl_profile.h); synchronises the device."""
+    import numpy as np
+    L = _profile_lib()
+    k, c, s = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    _check(L.kdkl_profile_role_cycles_shape(ctypes.byref(k), ctypes.byref(c), ctypes.byref(s)),
+           "kdkl_profile_role_cycles_shape")
+    out = np.zeros((k.value, c.value, s.value), dtype=np.uint64)
+    _check(L.kdkl_profile_read_role_cycles(out.ctypes.data, out.nbytes), "kdkl_profile_read_role_cycles")
+    return out
+
+
+def kdkl_profile_role_cycles_clear(stream=None) -> None:
+    """Zeroes the profiling build's role cycle counters on `stream`."""
+    _check(_profile_lib().kdkl_profile_clear_role_cycles(_stream(stream)), "kdkl_profile_clear_role_cycles")

@@ -9,6 +9,11 @@ TMA coordinate and lockstep slot is range-checked in the kernels, and a failed
 check sets ``KDKL_DEV_BOUNDS`` in the device flag word and skips (or clamps) the
 access instead of making it.  It stands in for a memory checker, which this
 hardware pool does not offer; the tests run the ragged parity cases through it.
+
+A third, ``_lib/libkdkl_prof.so``, is compiled with ``-DKDKL_PROFILE``: the same
+kernels, which also count the SM cycles their TMA producer, MMA issuer and
+epilogue spend at their barrier waits (``include/kdkl_profile.h``;
+``python -m output_head_kl_b200.profile_roles`` reports them).
 """
 from __future__ import annotations
 
@@ -22,6 +27,7 @@ CSRC = os.path.join(HERE, "csrc")
 OUT_DIR = os.path.join(HERE, "_lib")
 LIB = os.path.join(OUT_DIR, "libkdkl.so")
 DEBUG_LIB = os.path.join(OUT_DIR, "libkdkl_debug.so")
+PROFILE_LIB = os.path.join(OUT_DIR, "libkdkl_prof.so")
 SOURCES = ("kernels.cu", "api.cu", "noalloc.cu")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
@@ -41,6 +47,7 @@ def _stale(lib: str) -> bool:
     t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, f) for f in os.listdir(CSRC)]
     deps.append(os.path.join(os.path.dirname(HERE), "include", "kdkl.h"))
+    deps.append(os.path.join(os.path.dirname(HERE), "include", "kdkl_profile.h"))
     deps.append(os.path.abspath(__file__))
     return any(os.path.getmtime(p) > t for p in deps)
 
@@ -68,8 +75,9 @@ def _build_one(lib: str, prefix: str, defines, log_name: str):
     return logs
 
 
-def build(force: bool = False, verbose: bool = False, debug: bool = True) -> str:
-    """Builds libkdkl.so (and, with debug=True, the bounds-checking libkdkl_debug.so)."""
+def build(force: bool = False, verbose: bool = False, debug: bool = True, profile: bool = True) -> str:
+    """Builds libkdkl.so (and, when asked, the bounds-checking libkdkl_debug.so and the
+    cycle-counting libkdkl_prof.so)."""
     os.makedirs(OUT_DIR, exist_ok=True)
     if force or _stale(LIB):
         logs = _build_one(LIB, "", [], "ptxas.log")
@@ -77,6 +85,8 @@ def build(force: bool = False, verbose: bool = False, debug: bool = True) -> str
             print("\n".join(logs))
     if debug and (force or _stale(DEBUG_LIB)):
         _build_one(DEBUG_LIB, "dbg_", ["-DKDKL_DEBUG"], "ptxas_debug.log")
+    if profile and (force or _stale(PROFILE_LIB)):
+        _build_one(PROFILE_LIB, "prof_", ["-DKDKL_PROFILE"], "ptxas_prof.log")
     return LIB
 
 

@@ -132,6 +132,10 @@ struct EpiParams {
 // kEpiLseStore: the forward's online log-sum-exp and gather (as kEpiLse), and
 // every fp32 logit tile also stored to a chunk buffer (fused forward + backward).
 enum EpiKind { kEpiLse = 0, kEpiGrad = 1, kEpiStoreBf16 = 2, kEpiRmwF32 = 3, kEpiTopK = 4, kEpiLseStore = 5 };
+// Shape of the profiling build's role cycle counters: [epilogue kind][CTA][slot].
+constexpr int kRoleKinds = 8;
+constexpr int kRoleCtas = 256;
+constexpr int kRoleSlots = 12;
 
 // Teacher top-K producer: per-row min-heaps of up to kTopKMax entries live in
 // shared memory during the vocabulary sweep, with 16-bit indices relative to

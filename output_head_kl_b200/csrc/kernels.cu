@@ -483,6 +483,50 @@ __device__ int wait_split_peers(const Sched& sc, int u, int group, int ngroups, 
 }
 
 // z[off] for a run-time off in [0, 32) without dynamic register indexing.
+// Role cycle counters of the profiling build (-DKDKL_PROFILE).  Each GEMM CTA adds, under
+// its epilogue kind, how many SM cycles its TMA producer, its MMA issuer (the even CTA of
+// a pair) and its first epilogue warp spent in the kernel and waiting at their barriers:
+//   slots 0-3   MMA issuer: total, waiting for a free accumulator, waiting for operands, tiles
+//   slots 4-7   producer:   total, waiting for a free stage, waiting in the lockstep, units
+//   slots 8-11  epilogue:   total, waiting for a finished accumulator, 0, tiles
+// In every other build RoleClock is empty and compiles to nothing.
+#if defined(KDKL_PROFILE)
+__device__ unsigned long long g_role_cycles[kRoleKinds][kRoleCtas][kRoleSlots];
+
+__device__ __forceinline__ long long sm_cycles() {
+#if defined(__CUDA_ARCH__)
+  return clock64();
+#else
+  return 0;
+#endif
+}
+
+struct RoleClock {
+  long long start, w0 = 0, w1 = 0, n = 0;
+  __device__ RoleClock() : start(sm_cycles()) {}
+  __device__ long long now() const { return sm_cycles(); }
+  __device__ void wait0(long long t) { w0 += sm_cycles() - t; }
+  __device__ void wait1(long long t) { w1 += sm_cycles() - t; }
+  __device__ void count() { ++n; }
+  __device__ void flush(int kind, int base) const {
+    if (blockIdx.x >= static_cast<unsigned>(kRoleCtas) || kind >= kRoleKinds) return;
+    unsigned long long* p = g_role_cycles[kind][blockIdx.x] + base;
+    atomicAdd(p + 0, static_cast<unsigned long long>(sm_cycles() - start));
+    atomicAdd(p + 1, static_cast<unsigned long long>(w0));
+    atomicAdd(p + 2, static_cast<unsigned long long>(w1));
+    atomicAdd(p + 3, static_cast<unsigned long long>(n));
+  }
+};
+#else
+struct RoleClock {
+  __device__ long long now() const { return 0; }
+  __device__ void wait0(long long) {}
+  __device__ void wait1(long long) {}
+  __device__ void count() {}
+  __device__ void flush(int, int) const {}
+};
+#endif
+
 __device__ __forceinline__ float pick32(const float (&v)[32], uint32_t off) {
   float t16[16], t8[8], t4[4], t2[2];
   const bool b4 = off & 16u, b3 = off & 8u, b2 = off & 4u, b1 = off & 2u, b0 = off & 1u;
@@ -590,6 +634,7 @@ __global__ void __launch_bounds__(192, 1)
     int stage = 0;
     uint32_t phase = 0;
     bool wrapped = false;    // every stage has been filled at least once
+    RoleClock rc;
     bool stop = false;
     const bool sync_on = sc.sync_window > 0 && rank == 0;
     // row-stream units synchronise per tile; tile-mode units (one long reduction each)
@@ -600,6 +645,7 @@ __global__ void __launch_bounds__(192, 1)
     for (int u = group; u < sc.units && !stop; u += ngroups) {
       int mb, uj, t0, t1;
       unit_range(sc, u, mb, uj, t0, t1);
+      rc.count();
       const int arow = mb * C::kMmaM + static_cast<int>(rank) * kBM;   // this CTA's A rows
       bool hold = sync_on;
       int seen = -1;          // every peer had reached this position at the last look
@@ -615,7 +661,9 @@ __global__ void __launch_bounds__(192, 1)
             if (lane == 0) *reinterpret_cast<volatile unsigned long long*>(sc.prog + group) = sync_word(u, pos);
             __syncwarp();
             if (hold && need > seen) {
+              const long long c0 = rc.now();
               const int got = wait_split_peers(sc, u, group, ngroups, uj, need, lane, ep.flags);
+              rc.wait1(c0);
               if (got == -2) hold = false;
               else seen = got;
             }
@@ -624,7 +672,10 @@ __global__ void __launch_bounds__(192, 1)
           if (lane == 0) {
             const int kb1 = min(kb0 + kseg, sc.k_blocks);
             for (int kb = kb0; kb < kb1; ++kb) {
-              if (!mbar_wait(&empty[stage], phase ^ 1u, ab)) {
+              const long long c0 = rc.now();
+              const bool got_stage = mbar_wait(&empty[stage], phase ^ 1u, ab);
+              rc.wait0(c0);
+              if (!got_stage) {
                 lstop = 1;
                 break;
               }
@@ -690,6 +741,7 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
     }
+    if (lane == 0) rc.flush(KIND, 4);
     if (lane == 0 && rank == 0 && *abort_flag) {
       // The kernel is giving up: before shared memory is released, wait (bounded) until
       // the copies already issued have landed.  The even CTA's full barriers count
@@ -711,15 +763,23 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
+      RoleClock rc;
       for (int u = group; u < sc.units; u += ngroups) {
         int mb, uj, t0, t1;
         unit_range(sc, u, mb, uj, t0, t1);
         for (int t = t0; t < t1; ++t) {
-          if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, ab)) goto mma_done;
+          const long long c0 = rc.now();
+          const bool got_acc = mbar_wait(&acc_empty[acc], acc_phase ^ 1u, ab);
+          rc.wait0(c0);
+          rc.count();
+          if (!got_acc) goto mma_done;
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::kAccStride);
           for (int kb = 0; kb < sc.k_blocks; ++kb) {
-            if (!mbar_wait(&full[stage], phase, ab)) goto mma_done;
+            const long long c1 = rc.now();
+            const bool got_ops = mbar_wait(&full[stage], phase, ab);
+            rc.wait1(c1);
+            if (!got_ops) goto mma_done;
             tc_fence_after();
             const uint32_t a_addr = smem_u32(sA + stage * C::kABytes);
             const uint32_t b_addr = smem_u32(sB + stage * C::kBBytes);
@@ -746,6 +806,7 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
     mma_done:
+      rc.flush(KIND, 0);
       // every MMA issued above has finished before TMEM or shared memory is released
       if (PAIR) umma_commit_pair(drain, 0x1);
       else umma_commit(drain);
@@ -770,6 +831,7 @@ __global__ void __launch_bounds__(192, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     float g_scale = 0.f;
+    RoleClock rc;
     if (KIND == kEpiGrad) {
       // d loss / d z = (g / (tau_s N_valid)) (weight P_S - target)
       const uint32_t nv = *ep.n_valid;
@@ -836,7 +898,11 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       for (int t = t0; t < t1; ++t) {
-        if (!mbar_wait(&acc_full[acc], acc_phase, ab)) goto epi_done;
+        const long long c0 = rc.now();
+        const bool got_acc = mbar_wait(&acc_full[acc], acc_phase, ab);
+        rc.wait0(c0);
+        rc.count();
+        if (!got_acc) goto epi_done;
         tc_fence_after();
         const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(acc * C::kAccStride);
         // columns of this tile: [t * BN, col_lim); a last 32-column chunk that runs past
@@ -1101,6 +1167,7 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   epi_done:
+    if (q == 0 && lane == 0) rc.flush(KIND, 8);
     if (KIND == kEpiRmwF32 && lane == 0 && dw_pending) {
       // a load of an old dW block may still be landing (abort path): bounded wait
       const uint64_t w0 = globaltimer_ns();
@@ -1517,3 +1584,30 @@ cudaError_t launch_topk_merge(const float* part_tv, const int* part_ti, int spli
 }
 
 }  // namespace kdkl
+
+#if defined(KDKL_PROFILE)
+// Host side of the role cycle counters (declared in kdkl_profile.h).
+#include "../../include/kdkl_profile.h"
+
+extern "C" kdkl_status kdkl_profile_role_cycles_shape(int32_t* kinds, int32_t* ctas, int32_t* slots) {
+  if (!kinds || !ctas || !slots) return KDKL_ERR_NULL;
+  *kinds = kdkl::kRoleKinds;
+  *ctas = kdkl::kRoleCtas;
+  *slots = kdkl::kRoleSlots;
+  return KDKL_OK;
+}
+
+extern "C" kdkl_status kdkl_profile_read_role_cycles(void* host_dst, size_t bytes) {
+  if (!host_dst) return KDKL_ERR_NULL;
+  if (bytes != sizeof(kdkl::g_role_cycles)) return KDKL_ERR_SHAPE;
+  return cudaMemcpyFromSymbol(host_dst, kdkl::g_role_cycles, bytes) == cudaSuccess ? KDKL_OK : KDKL_ERR_CUDA;
+}
+
+extern "C" kdkl_status kdkl_profile_clear_role_cycles(void* stream) {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, kdkl::g_role_cycles) != cudaSuccess) return KDKL_ERR_CUDA;
+  return cudaMemsetAsync(p, 0, sizeof(kdkl::g_role_cycles), static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? KDKL_OK
+             : KDKL_ERR_CUDA;
+}
+#endif
