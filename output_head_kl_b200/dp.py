@@ -10,7 +10,11 @@ replica of the output-head weight W.  One step:
    global loss, and an all-reduce (sum) gives the global loss;
 3. backward on the shard with the same normaliser, so the local dW is this
    shard's term of the global gradient and dHidden is already final;
-4. all-reduce dW (sum), the one real exchange of the step.
+4. all-reduce dW (sum), the one real exchange of the step; with ``dw_buckets`` > 1
+   it runs as that many asynchronous collectives over contiguous slices of
+   vocabulary rows, so that a caller who leaves them pending (``wait_dw=False``)
+   can update each slice of W as soon as its reduction completes while the later
+   slices are still in flight.
 
 All arithmetic of the loss and its normalisation runs in the library; this
 module only issues the library calls and the collectives.  `ops` abstracts the
@@ -30,8 +34,10 @@ class StepResult:
     loss: torch.Tensor        # [1] global loss (identical on every rank)
     lse: torch.Tensor         # [N_local]
     dHidden: torch.Tensor     # [N_local, d]
-    dW: torch.Tensor          # [V, d], all-reduced
+    dW: torch.Tensor          # [V, d], all-reduced (once dw_work has completed)
     n_valid_global: torch.Tensor
+    # pending (row slice, work) pairs of dW's reduction when dp_step(wait_dw=False)
+    dw_work: list = dataclasses.field(default_factory=list)
 
 
 class KernelOps:
@@ -74,7 +80,23 @@ class KernelOps:
         return dH, dW
 
 
-def dp_step(hidden, W, topk_idx, topk_logit, mask, tau, *, ops=None, group=None) -> StepResult:
+def allreduce_dw_buckets(dW, buckets: int, group=None) -> list:
+    """Starts the sum all-reduce of dW as `buckets` asynchronous collectives over
+    contiguous slices of its rows (vocabulary entries), and returns the (row slice, work)
+    pairs in row order.  Each element is still summed over the same ranks by one
+    collective, so the result equals a single all-reduce of the whole tensor up to the
+    order in which the ranks' terms are added (exactly, with two ranks)."""
+    V = dW.shape[0]
+    buckets = max(1, min(int(buckets), V)) if V else 1
+    out = []
+    for b in range(buckets):
+        rows = slice(b * V // buckets, (b + 1) * V // buckets)
+        out.append((rows, dist.all_reduce(dW[rows], op=dist.ReduceOp.SUM, group=group, async_op=True)))
+    return out
+
+
+def dp_step(hidden, W, topk_idx, topk_logit, mask, tau, *, ops=None, group=None, dw_buckets: int = 1,
+            wait_dw: bool = True) -> StepResult:
     """One token-sharded data-parallel forward + backward (see the module docstring)."""
     ops = ops or KernelOps()
     world = dist.get_world_size(group) if dist.is_initialized() else 1
@@ -86,6 +108,14 @@ def dp_step(hidden, W, topk_idx, topk_logit, mask, tau, *, ops=None, group=None)
     if world > 1:
         dist.all_reduce(loss, op=dist.ReduceOp.SUM, group=group)
     dH, dW = ops.backward(hidden, W, topk_idx, topk_logit, mask, tau, lse, ws, total)
+    work = []
     if world > 1:
-        dist.all_reduce(dW, op=dist.ReduceOp.SUM, group=group)
-    return StepResult(loss, lse, dH, dW, total)
+        if dw_buckets > 1:
+            work = allreduce_dw_buckets(dW, dw_buckets, group)
+        else:
+            dist.all_reduce(dW, op=dist.ReduceOp.SUM, group=group)
+    if wait_dw:
+        for _, w in work:
+            w.wait()
+        work = []
+    return StepResult(loss, lse, dH, dW, total, work)

@@ -83,3 +83,50 @@ def test_dp_step_equals_single_process():
     np.testing.assert_allclose(dW0, full.dW, rtol=1e-12, atol=1e-18)
     np.testing.assert_array_equal(dW0, dW1)
     np.testing.assert_allclose(np.concatenate([dH0, dH1]), full.dH, rtol=1e-12, atol=1e-18)
+
+
+def _bucket_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        g = torch.Generator().manual_seed(1000 + rank)
+        base = torch.randn(101, 16, generator=g, dtype=torch.float32)
+        whole = base.clone()
+        dist.all_reduce(whole)
+        res = {}
+        for buckets in (1, 3, 7, 500):
+            t = base.clone()
+            work = dp.allreduce_dw_buckets(t, buckets)
+            slices = [sl for sl, _ in work]
+            for _, w in work:
+                w.wait()
+            res[buckets] = (t.numpy().copy(), [(sl.start, sl.stop) for sl in slices])
+        # the step itself, with the reduction left pending and then completed by the caller
+        x = synth.custom_inputs(37, 16, 101, 6, seed=81, mask_frac=0.2, w_std=0.3)
+        s = _shard(x, rank, world)
+        one = dp.dp_step(None, None, None, None, None, x.tau, ops=OracleOps(s))
+        pend = dp.dp_step(None, None, None, None, None, x.tau, ops=OracleOps(s), dw_buckets=4, wait_dw=False)
+        n_pending = len(pend.dw_work)
+        for _, w in pend.dw_work:
+            w.wait()
+        out[rank] = (whole.numpy().copy(), res, one.dW.numpy().copy(), pend.dW.numpy().copy(), n_pending)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bucketed_dw_reduction_equals_one_all_reduce():
+    """dW reduced in slices of vocabulary rows (asynchronous collectives, one per slice)
+    equals one all-reduce of the whole tensor; the slices partition the rows in order; and
+    a step that leaves the slices pending gives the same dW once the caller waits."""
+    out = mp.get_context("spawn").Manager().dict()
+    mp.start_processes(_bucket_worker, args=(2, _port(), out), nprocs=2, join=True, start_method="spawn")
+    for rank in (0, 1):
+        whole, res, dw_one, dw_pend, n_pending = out[rank]
+        for buckets, (t, slices) in res.items():
+            np.testing.assert_array_equal(t, whole, err_msg=f"buckets={buckets}")
+            assert slices[0][0] == 0 and slices[-1][1] == 101
+            assert all(a[1] == b[0] for a, b in zip(slices, slices[1:]))
+            assert len(slices) == min(buckets, 101)
+        assert n_pending == 4
+        np.testing.assert_array_equal(dw_pend, dw_one)
+    np.testing.assert_array_equal(out[0][0], out[1][0])
