@@ -5,7 +5,9 @@ batch with gloo collectives (the exchanges pass through the host; no kernel
 waits on the other rank).  The result must be the single-process step on the
 whole batch: the same valid count and loss on both ranks, the same all-reduced
 dW on both ranks (bit for bit) and equal to the whole-batch dW, and each
-rank's dHidden rows equal to the whole-batch rows.  Per-row results can differ
+rank's dHidden rows equal to the whole-batch rows.  dW reduced in slices of
+vocabulary rows, left pending by the step and completed by the caller, must equal
+the one-collective dW bit for bit.  Per-row results can differ
 from the whole-batch run only by rounding, because the forward's vocabulary
 split count (and so the order of its log-sum-exp merge) depends on the batch
 size.
@@ -42,9 +44,11 @@ def _half(x, rank):
     return synth.Inputs(x.hidden_bits[sl], x.W_bits, x.topk_idx[sl], x.topk_logit[sl], x.mask[sl], x.tau)
 
 
-def _step(x):
+def _step(x, **kw):
     d = H.to_device(x)
-    r = dp.dp_step(d.hidden, d.W, d.idx, d.logit, d.mask, d.tau)
+    r = dp.dp_step(d.hidden, d.W, d.idx, d.logit, d.mask, d.tau, **kw)
+    for _, w in r.dw_work:       # a bucketed reduction left pending: the caller completes it
+        w.wait()
     torch.cuda.synchronize()
     return (float(r.loss.item()), r.dW.cpu().numpy().astype(np.float64), r.dHidden.float().cpu().numpy(),
             int(r.n_valid_global.item()))
@@ -56,6 +60,8 @@ def _worker(rank, world, port, out):
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
     try:
         out[rank] = _step(_half(_inputs(), rank))
+        # dW reduced in 5 slices of vocabulary rows, left pending by the step
+        out[10 + rank] = _step(_half(_inputs(), rank), dw_buckets=5, wait_dw=False)[1]
     finally:
         dist.destroy_process_group()
 
@@ -76,6 +82,8 @@ def test_two_ranks_equal_one_process():
     assert l0 == l1
     assert abs(l0 - loss) <= 1e-5 * abs(loss)
     np.testing.assert_array_equal(dW0, dW1)
+    np.testing.assert_array_equal(out[10], dW0)   # the bucketed reduction gives the same dW
+    np.testing.assert_array_equal(out[11], dW1)
     assert np.abs(dW0 - dW).max() <= 1e-3 * np.abs(dW).max()
     dH_ranks = np.concatenate([dH0, dH1])
     assert np.abs(dH_ranks - dH).max() <= 1e-3 * np.abs(dH).max()
