@@ -1,11 +1,13 @@
 """Where the GEMM kernels' cycles go: the profiling build's role counters.
 
-    python -m output_head_kl_b200.profile_roles --config 8b [--N n] [--phase step|fused|topk] [--reps r]
+    python -m output_head_kl_b200.profile_roles --config 8b [--N n] [--phase step|bwd|fused|topk] [--reps r]
+                                                [--chunk-tokens c] [--bwd-tile-n w]
 
 Loads ``_lib/libkdkl_prof.so`` (the library compiled with ``-DKDKL_PROFILE``, whose
 GEMM CTAs count the SM cycles their roles spend at barrier waits, see
 ``include/kdkl_profile.h``), runs the phase ``--warmup`` times, clears the counters,
-runs it ``--reps`` times and prints one JSON line.  Per GEMM kind:
+runs it ``--reps`` times and prints one JSON line (``bwd``: one untimed forward, then
+the backward alone; ``--bwd-tile-n`` forces the dHidden / dW tile width).  Per GEMM kind:
 
 * ``flops_per_sm_cycle``: the kind's dense flops (2·N·d·V per launch set) over the
   SM cycles of its CTAs (each MMA issuer's cycles times the CTAs it issues for); the
@@ -73,7 +75,9 @@ def main(argv=None) -> int:
     ap = argparse.ArgumentParser()
     ap.add_argument("--config", default="8b", choices=sorted(synth.CONFIGS))
     ap.add_argument("--N", type=int, default=None)
-    ap.add_argument("--phase", default="step", choices=["step", "fused", "topk"])
+    ap.add_argument("--phase", default="step", choices=["step", "bwd", "fused", "topk"])
+    ap.add_argument("--chunk-tokens", type=int, default=0)
+    ap.add_argument("--bwd-tile-n", type=int, default=0)
     ap.add_argument("--warmup", type=int, default=2)
     ap.add_argument("--reps", type=int, default=1)
     a = ap.parse_args(argv)
@@ -104,17 +108,30 @@ def main(argv=None) -> int:
         lse = torch.empty(N, dtype=torch.float32, device=dev)
         dH = torch.empty(N, d, dtype=torch.bfloat16, device=dev)
         dW = torch.empty(V, d, dtype=torch.float32, device=dev)
+        opts = K.kdkl_options(bwd_tile_n=a.bwd_tile_n)
+        ch = a.chunk_tokens
         if a.phase == "fused":
-            ws = torch.empty(K.kdkl_forward_backward_workspace_bytes(N, d, V, Kc, 0), dtype=torch.uint8, device=dev)
+            ws = torch.empty(K.kdkl_forward_backward_workspace_bytes(N, d, V, Kc, ch), dtype=torch.uint8, device=dev)
 
             def run():
-                K.kdkl_forward_backward(hidden, W, idx, logit, mask, x.tau, loss, lse, dH, dW, ws)
+                K.kdkl_forward_backward(hidden, W, idx, logit, mask, x.tau, loss, lse, dH, dW, ws, opts,
+                                        chunk_tokens=ch)
         else:
-            ws = torch.empty(K.kdkl_workspace_bytes(N, d, V, Kc, 0), dtype=torch.uint8, device=dev)
+            ws = torch.empty(K.kdkl_workspace_bytes(N, d, V, Kc, ch), dtype=torch.uint8, device=dev)
 
-            def run():
-                K.kdkl_forward(hidden, W, idx, logit, mask, x.tau, loss, lse, ws)
-                K.kdkl_backward(hidden, W, idx, logit, mask, x.tau, lse, None, dH, dW, ws)
+            def fwd():
+                K.kdkl_forward_ex(hidden, W, idx, logit, mask, x.tau, loss, lse, ws, opts)
+
+            def bwd():
+                K.kdkl_backward_ex(hidden, W, idx, logit, mask, x.tau, lse, None, dH, dW, ws, opts, chunk_tokens=ch)
+
+            if a.phase == "bwd":
+                fwd()
+                run = bwd
+            else:
+                def run():
+                    fwd()
+                    bwd()
 
     for _ in range(a.warmup):
         run()
@@ -129,6 +146,7 @@ def main(argv=None) -> int:
     counters = K.kdkl_profile_role_cycles_read()
     flags = K.kdkl_read_device_flags(ws)
     rec = {"workload": w.name, "N": N, "d": d, "V": V, "K": Kc, "phase": a.phase, "reps": a.reps,
+           "chunk_tokens": a.chunk_tokens, "bwd_tile_n": a.bwd_tile_n,
            "ms_per_rep": e0.elapsed_time(e1) / a.reps, "device_flags": flags,
            "kinds": summarise(counters, 2.0 * N * d * V * a.reps)}
     print(json.dumps(rec), flush=True)
